@@ -1,0 +1,100 @@
+"""Planted mistakes in the oracle (on the CPU) must each fail a pin.
+
+These show that the pins in ``test_oracle_pins.py`` are sensitive to the
+mistakes an fp64 restatement of the block is likely to contain.
+"""
+import math
+import types
+
+import numpy as np
+import pytest
+
+import oracle
+import oracle.tp_block as tb
+from tests import test_oracle_pins as pins
+
+
+def _expect_fail(check):
+    with pytest.raises(AssertionError):
+        check()
+
+
+def test_tanh_gelu_is_caught(monkeypatch):
+    # the tanh approximation written as an erf replacement: erf(u) ~ tanh(c (x + 0.044715 x^3)), x = u sqrt 2
+    def erf_tanh(u):
+        x = np.asarray(u) * math.sqrt(2.0)
+        return np.tanh(math.sqrt(2.0 / math.pi) * (x + 0.044715 * x ** 3))
+    monkeypatch.setattr(tb, "_erf", erf_tanh)
+    _expect_fail(pins.check_gelu_table)
+
+
+def test_wrong_attention_scale_is_caught(monkeypatch):
+    fake_math = types.SimpleNamespace(sqrt=lambda x: float(x))  # 1/d instead of 1/sqrt(d)
+    monkeypatch.setattr(tb, "math", fake_math)
+    _expect_fail(pins.check_attention_core)
+
+
+def test_off_by_one_causal_mask_is_caught(monkeypatch):
+    def attention_strict(Q, K, V, causal, q_pos=None):
+        Q, K, V = (np.asarray(a, float) for a in (Q, K, V))
+        nq, Hn, d = Q.shape
+        S = K.shape[0]
+        q_pos = np.arange(nq) if q_pos is None else np.asarray(q_pos)
+        keep = (np.arange(S)[None, :] < q_pos[:, None] + (0 if causal else S))
+        keep[:, 0] = True  # keeps row 0 finite; the mistake is j < i elsewhere
+        O = np.empty((nq, Hn, d))
+        for g in range(Hn):
+            s = np.where(keep, Q[:, g] @ K[:, g].T / math.sqrt(d), -np.inf)
+            p = np.exp(s - s.max(1, keepdims=True))
+            O[:, g] = (p / p.sum(1, keepdims=True)) @ V[:, g]
+        return O
+    monkeypatch.setattr(oracle, "attention_heads", attention_strict)
+    monkeypatch.setattr(tb, "attention_heads", attention_strict)
+    _expect_fail(pins.check_attention_core)
+
+
+def test_unbiased_variance_is_caught(monkeypatch):
+    def ln_unbiased(x, g, b, eps=1e-5):
+        x = np.asarray(x, float)
+        mu = x.mean(-1, keepdims=True)
+        var = x.var(-1, ddof=1, keepdims=True)
+        y = (x - mu) / np.sqrt(var + eps)
+        return y * (1 if g is None else g) + (0 if b is None else b)
+    monkeypatch.setattr(oracle, "layernorm", ln_unbiased)
+    monkeypatch.setattr(tb, "layernorm", ln_unbiased)
+    _expect_fail(pins.check_layernorm)
+
+
+def test_bias_per_shard_is_caught(monkeypatch):
+    real = tb.ffn_forward_sharded
+
+    def b2_per_shard(X, shards, b2, R, act="gelu"):
+        shards = list(shards)
+        return real(X, shards, None if b2 is None else np.asarray(b2) * len(shards), R, act)
+    monkeypatch.setattr(oracle, "ffn_forward_sharded", b2_per_shard)
+    _expect_fail(pins.check_ffn_sharding_invariance)
+
+
+def test_dropped_residual_is_caught(monkeypatch):
+    real = tb.ffn_forward
+
+    def no_residual(X, W1, b1, W2, b2, R, act="gelu"):
+        return real(X, W1, b1, W2, b2, None, act)
+    monkeypatch.setattr(oracle, "ffn_forward", no_residual)
+    _expect_fail(pins.check_ffn_brute_force)
+
+
+def test_transposed_wo_is_caught(monkeypatch):
+    real = tb.attn_forward
+
+    def wo_transposed(X, Wq, Wk, Wv, Wo, bo, R, B, S, H, d, causal=True, rows=None, bqkv=None):
+        return real(X, Wq, Wk, Wv, np.asarray(Wo).T, bo, R, B, S, H, d, causal, rows, bqkv)
+    monkeypatch.setattr(oracle, "attn_forward", wo_transposed)
+    _expect_fail(pins.check_attention_sharding_and_heads)
+
+
+def test_missing_layernorm_in_layer_is_caught(monkeypatch):
+    def identity_ln(x, g, b, eps=1e-5):
+        return np.asarray(x, float)
+    monkeypatch.setattr(tb, "layernorm", identity_ln)
+    _expect_fail(pins.check_layer)
