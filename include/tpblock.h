@@ -1,0 +1,218 @@
+/*
+ * libtpblock -- the Megatron column->row tensor-parallel transformer block,
+ * forward pass, on one B200 (sm_100a).
+ *
+ * Source of the method: "Tensor Parallelism > Combining Column and Row
+ * Parallelism" (mbrenndoerfer.com), cited below as [TP-CR]:
+ *   step 1  column-parallel W1: shard i computes Z_i = X W1_i, then GeLU(Z_i),
+ *           with no communication;
+ *   step 2  row-parallel W2: Y_i = GeLU(Z_i) W2_i, a partial sum over the
+ *           full output;
+ *   step 3  all-reduce: Y = sum_i Y_i;
+ *   and the paragraphs on multi-head attention (QKV column-parallel by head
+ *   group, output projection row-parallel), on feature reductions (LayerNorm
+ *   needs the full row) and on the two reductions per layer with residual
+ *   adds between the sub-layers.
+ *
+ * All t logical shards run on the one GPU; step 3 becomes an on-device
+ * reduction (fixed order i = 0..t-1, no atomics, bitwise reproducible).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Pointers are DEVICE pointers unless stated otherwise.  The caller owns
+ *    every buffer, including the workspace; the library never allocates,
+ *    frees or synchronises (except tp_get_device_status, which synchronises
+ *    the given stream).
+ *  - Matrices are row-major.  A tp_shard is a view {ptr, ld}: element (r, c)
+ *    is at ptr + r*ld + c (ld in elements).  Shards may point into one big
+ *    matrix (e.g. W1_i = W1 + i*f/t with ld = f) or into separate buffers.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream).  Launches go to that stream only.
+ *  - Host validation runs before any launch.  On failure the call returns
+ *    TP_ERR_INVALID_ARG or TP_ERR_UNSUPPORTED, launches nothing, and
+ *    tp_last_error() describes the failed check.  A failed launch returns
+ *    TP_ERR_CUDA.  A device-side wait that runs past its time limit makes the
+ *    kernel stop, and tp_get_device_status() then returns TP_ERR_TIMEOUT.
+ *  - bf16 paths: element type IEEE bfloat16, fp32 accumulation, results
+ *    rounded to nearest even.  Every bf16 pointer must be 16-byte aligned,
+ *    every ld a multiple of 8, and h, f/t and (heads/t)*d multiples of 64.
+ *  - Stateless and thread-safe apart from the optional launch trace.
+ */
+#ifndef TPBLOCK_H
+#define TPBLOCK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define TP_API __attribute__((visibility("default")))
+#else
+#define TP_API
+#endif
+
+#define TP_MAX_SHARDS 16
+
+typedef enum {
+  TP_OK = 0,
+  TP_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer or ld */
+  TP_ERR_UNSUPPORTED = 2, /* valid but outside what the kernels implement */
+  TP_ERR_WORKSPACE = 3,   /* workspace missing or smaller than *_workspace_bytes */
+  TP_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+  TP_ERR_TIMEOUT = 5      /* a device wait ran out (reported by tp_get_device_status) */
+} tp_status;
+
+typedef enum { TP_BF16 = 0, TP_FP32 = 1 } tp_dtype;
+
+/* How step 3 (the all-reduce) is done on one device.
+ * TP_REDUCE_FUSED:    one row-GEMM tile accumulates the K-slices of all t
+ *                     shards in order into one fp32 accumulator, and its
+ *                     epilogue adds the bias and the residual.
+ * TP_REDUCE_PARTIALS: the row GEMM writes t fp32 partials Y_i [t, M, h] to the
+ *                     workspace; a reduce kernel sums them in order 0..t-1
+ *                     and adds bias and residual. */
+typedef enum { TP_REDUCE_FUSED = 0, TP_REDUCE_PARTIALS = 1 } tp_reduce_mode;
+
+/* Element-wise nonlinearity of step 1: exact GeLU z*Phi(z) (erf form) or ReLU. */
+typedef enum { TP_ACT_GELU = 0, TP_ACT_RELU = 1 } tp_activation;
+
+typedef struct {
+  const void* ptr; /* device pointer to element (0, 0) of the shard */
+  int64_t ld;      /* row stride in elements */
+} tp_shard;
+
+typedef void* tp_stream_t; /* cudaStream_t */
+
+/* ------------------------------------------------------------------ FFN block
+ * [TP-CR] steps 1-3:  out = sum_{i<t} act(X W1_i + b1_i) W2_i + b2 + residual.
+ *
+ *  X        [M, h], dtype, ld = h (contiguous).
+ *  W1[i]    [h, f/t] view, i < t (column shard i of W1 [h, f]).
+ *  b1       array of t pointers to [f/t] vectors, or NULL (no bias).
+ *  W2[i]    [f/t, h] view (row shard i of W2 [f, h]).
+ *  b2       [h] or NULL; added once, after the sum over shards.
+ *  residual [M, h] or NULL; added after the sum (may alias X).
+ *  out      [M, h], contiguous; must not alias X, residual or the weights.
+ *  dtype    TP_BF16 (tensor cores) or TP_FP32 (exact fp32 FFMA, no TF32).
+ *  mode     see tp_reduce_mode (ignored for TP_FP32, which always uses partials).
+ *  ws       device workspace of at least tp_ffn_workspace_bytes(...) bytes,
+ *           256-byte aligned.  Holds act(Z) [M, f] (and the partials in
+ *           TP_REDUCE_PARTIALS mode).  Its contents on entry are ignored.
+ * Limits: 1 <= t <= TP_MAX_SHARDS, f % t == 0, M >= 1.
+ */
+TP_API size_t tp_ffn_workspace_bytes(int64_t M, int64_t h, int64_t f, int t, tp_dtype dtype, tp_reduce_mode mode);
+
+TP_API tp_status tp_ffn_forward(const void* X, int64_t M, int64_t h, int64_t f, int t, const tp_shard* W1,
+                         const void* const* b1, const tp_shard* W2, const void* b2, const void* residual,
+                         void* out, tp_dtype dtype, tp_reduce_mode mode, void* ws, size_t ws_bytes,
+                         tp_stream_t stream);
+
+/* Same block with a chosen nonlinearity ([TP-CR], the paragraph on where the
+ * nonlinearity fits: "GeLU (or ReLU)"). */
+TP_API tp_status tp_ffn_forward_act(const void* X, int64_t M, int64_t h, int64_t f, int t, const tp_shard* W1,
+                             const void* const* b1, const tp_shard* W2, const void* b2, const void* residual,
+                             void* out, tp_dtype dtype, tp_reduce_mode mode, tp_activation act, void* ws,
+                             size_t ws_bytes, tp_stream_t stream);
+
+/* ------------------------------------------------------------------ parallel linears
+ * Column-parallel linear alone ([TP-CR] step 1), bf16:
+ *   out[:, i*n/t : (i+1)*n/t] = act(X W_i + b_i)   for i < t,
+ *   X [M, k] contiguous, W[i] [k, n/t] views, b NULL or t pointers to [n/t],
+ *   out [M, n] contiguous bf16.  act: -1 = identity, else tp_activation. */
+TP_API tp_status tp_column_linear_forward(const void* X, int64_t M, int64_t k, int64_t n, int t, const tp_shard* W,
+                                   const void* const* b, int act, void* out, tp_stream_t stream);
+
+/* Row-parallel linear with the reduction ([TP-CR] steps 2-3), bf16:
+ *   out = sum_{i<t} A[:, i*k/t : (i+1)*k/t] W_i + bias + residual,
+ *   A [M, k] contiguous (the column layer's output), W[i] [k/t, n] views,
+ *   bias [n] or NULL, residual [M, n] or NULL, out [M, n] bf16.
+ *   ws: tp_row_linear_workspace_bytes(...) bytes (0 in TP_REDUCE_FUSED mode). */
+TP_API size_t tp_row_linear_workspace_bytes(int64_t M, int64_t n, int t, tp_reduce_mode mode);
+TP_API tp_status tp_row_linear_forward(const void* A, int64_t M, int64_t k, int64_t n, int t, const tp_shard* W,
+                                const void* bias, const void* residual, void* out, tp_reduce_mode mode, void* ws,
+                                size_t ws_bytes, tp_stream_t stream);
+
+/* ------------------------------------------------------------------ attention sub-layer
+ * [TP-CR], paragraphs on multi-head attention and head independence: the QKV
+ * projection is column-parallel by head group, each group attends over its
+ * own heads, the output projection is row-parallel and its partial sums are
+ * reduced:
+ *   out = sum_{i<t} O_i Wo_i + bo + residual,
+ *   O_i = concat over heads g of group i of softmax(Q_g K_g^T / sqrt(d) + mask) V_g.
+ *
+ *  X        [B*S, h] bf16 contiguous (row r = b*S + s).
+ *  Wqkv[i]  [h, 3*Hg*d] view, Hg = heads/t: columns [Q heads | K heads | V heads]
+ *           of group i, head g of the group at columns g*d .. g*d+d-1 of each block.
+ *  bqkv     NULL or t pointers to [3*Hg*d] bf16.
+ *  Wo[i]    [Hg*d, h] view (rows of the output projection for group i's heads).
+ *  bo       [h] or NULL.  residual [B*S, h] or NULL.  out [B*S, h] bf16.
+ *  causal   1: key j is visible to query i iff j <= i (same sequence); 0: all keys.
+ * Limits: d == 128, heads % t == 0, S >= 1.
+ */
+TP_API size_t tp_attn_workspace_bytes(int B, int S, int h, int heads, int d, int t, tp_reduce_mode mode);
+TP_API tp_status tp_attn_forward(const void* X, int B, int S, int h, int heads, int d, int t, const tp_shard* Wqkv,
+                          const void* const* bqkv, const tp_shard* Wo, const void* bo, const void* residual,
+                          int causal, void* out, tp_reduce_mode mode, void* ws, size_t ws_bytes,
+                          tp_stream_t stream);
+
+/* ------------------------------------------------------------------ pre-LN layer
+ * [TP-CR], the paragraph on two reductions per layer, in pre-LN order:
+ *   h1  = X + Attn(LN1(X))            (h1 kept in fp32 inside the workspace)
+ *   out = h1 + FFN(LN2(h1))           (bf16)
+ * LayerNorm runs replicated over the full row ([TP-CR], feature reductions).
+ * Weights as in tp_attn_forward and tp_ffn_forward; ln*_g / ln*_b are [h] bf16.
+ */
+TP_API size_t tp_layer_workspace_bytes(int B, int S, int h, int heads, int d, int64_t f, int t, tp_reduce_mode mode);
+TP_API tp_status tp_layer_forward(const void* X, int B, int S, int h, int heads, int d, int64_t f, int t,
+                           const void* ln1_g, const void* ln1_b, const tp_shard* Wqkv, const void* const* bqkv,
+                           const tp_shard* Wo, const void* bo, const void* ln2_g, const void* ln2_b,
+                           const tp_shard* W1, const void* const* b1, const tp_shard* W2, const void* b2, float eps,
+                           int causal, void* out, tp_reduce_mode mode, void* ws, size_t ws_bytes,
+                           tp_stream_t stream);
+
+/* ------------------------------------------------------------------ building blocks
+ * LayerNorm over rows: y = (x - mean) / sqrt(var + eps) * gamma + beta, var the
+ * biased variance.  x [M, h] bf16 or fp32 (in_dtype); gamma, beta [h] bf16 or
+ * NULL (1 and 0); y [M, h] bf16.  h % 8 == 0. */
+TP_API tp_status tp_layernorm_forward(const void* x, tp_dtype in_dtype, const void* gamma, const void* beta, int64_t M,
+                               int64_t h, float eps, void* y, tp_stream_t stream);
+
+/* Step 3 alone: out = sum_{i<t} P[i] + bias + residual in fixed order i = 0..t-1.
+ * P [t, M, h] fp32 contiguous; bias [h] and residual [M, h] in `dtype` or NULL;
+ * out [M, h] in `dtype`.  h % 4 == 0. */
+TP_API tp_status tp_reduce_partials(const float* P, int t, int64_t M, int64_t h, const void* bias, const void* residual,
+                             tp_dtype dtype, void* out, tp_stream_t stream);
+
+/* ------------------------------------------------------------------ status, limits, tracing */
+/* Synchronise `stream`, then read and clear the device status word of the
+ * current device.  TP_ERR_TIMEOUT if a device wait ran out since the last call;
+ * TP_ERR_CUDA if the synchronisation itself failed. */
+TP_API tp_status tp_get_device_status(tp_stream_t stream);
+
+/* Time limit of every device-side wait, in nanoseconds (default 2e9). */
+TP_API void tp_set_wait_limit_ns(uint64_t ns);
+
+/* Launch a one-CTA kernel that waits on a barrier nothing ever completes, with
+ * the given limit.  It must return and leave TP_ERR_TIMEOUT in the status word. */
+TP_API tp_status tp_selftest_bounded_wait(uint64_t limit_ns, tp_stream_t stream);
+
+/* Optional launch trace of the calling thread: while enabled, each kernel the
+ * library launches is bracketed by two CUDA events on its stream (at most
+ * `capacity` launches are kept).  After synchronising, tp_trace_get returns the
+ * kernel name and its event-timed duration in ms. */
+TP_API tp_status tp_trace_enable(int capacity);
+TP_API void tp_trace_disable(void);
+TP_API int tp_trace_count(void);
+TP_API tp_status tp_trace_get(int i, const char** name, float* ms);
+
+TP_API const char* tp_status_string(tp_status s);
+TP_API const char* tp_last_error(void);
+TP_API int tp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TPBLOCK_H */

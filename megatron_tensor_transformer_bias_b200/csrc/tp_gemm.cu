@@ -1,0 +1,376 @@
+// Persistent warp-specialised tcgen05 GEMM for the column- and row-parallel linears.
+//
+//   C_g[M, N] = A[:, g*a_k_per_group : +Kg] (M x Kg, K-major) * B_g (Kg x N, N-major)
+//
+// Column-parallel layer ("Tensor Parallelism > Combining Column and Row
+// Parallelism", step 1): one tile per (shard g, m-block, n-block); the
+// epilogue adds the shard's bias and applies the element-wise nonlinearity
+// straight from TMEM (no communication is needed, the nonlinearity is local).
+// Row-parallel layer (steps 2-3): either one tile per (m-block, n-block) whose
+// K loop walks the K-slices of shards 0..t-1 in order into the same TMEM
+// accumulator (the reduction happens in the accumulator) with a bias + residual
+// epilogue, or one tile per (shard, m, n) writing fp32 partials.
+//
+// Roles per CTA (192 threads, one CTA per SM):
+//   warp 0      TMA producer: A tile 128x64 and B tile 64x256 per stage
+//   warp 1      TMEM allocation; one thread issues tcgen05.mma (M=128, N=256, K=16)
+//   warps 2..5  epilogue: tcgen05.ld TMEM -> registers -> bias/act/residual -> global
+// A 4-stage shared-memory ring feeds the MMA; two 256-column TMEM accumulators let
+// the epilogue of one tile overlap the main loop of the next.
+#include "tp_internal.h"
+#include "tp_ptx.cuh"
+
+namespace tpb {
+
+namespace {
+
+constexpr int BM = GEMM_BM, BN = GEMM_BN, BK = GEMM_BK;
+constexpr int STAGES = 4;
+constexpr int A_STAGE_BYTES = BM * BK * 2;          // 16 KB
+constexpr int B_BLOCK_BYTES = 64 * BK * 2;          // 8 KB: 64 N-columns x 64 K-rows
+constexpr int B_STAGE_BYTES = BN * BK * 2;          // 32 KB
+constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+constexpr int NUM_ACC = 2;
+constexpr int TMEM_COLS = NUM_ACC * BN;             // 512
+constexpr int THREADS = 192;
+constexpr int EPI_THREADS = 128;
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, /*a_mn=*/0, /*b_mn=*/1);
+
+struct TileCoord {
+  int g, m_blk, n_blk;
+};
+
+__device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int tile, int m_tiles, int n_tiles) {
+  TileCoord c;
+  c.m_blk = tile % m_tiles;
+  const int rest = tile / m_tiles;
+  c.n_blk = rest % n_tiles;
+  c.g = a.concat ? 0 : rest / n_tiles;
+  return c;
+}
+
+__device__ __forceinline__ float act_apply(float v, int act) {
+  if (act == ACT_GELU) return v * 0.5f * (1.0f + erff(v * 0.70710678118654752440f));
+  if (act == ACT_RELU) return fmaxf(v, 0.0f);
+  return v;
+}
+
+__device__ __forceinline__ void load_bf16x32(const void* p, float (&v)[32]) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint4 u = __ldg(q + i);
+    uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[i * 8 + j * 2] = __uint_as_float(w[j] << 16);
+      v[i * 8 + j * 2 + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    }
+  }
+}
+
+__device__ __forceinline__ void load_f32x32(const void* p, float (&v)[32]) {
+  const float4* q = reinterpret_cast<const float4*>(p);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float4 u = __ldg(q + i);
+    v[i * 4] = u.x; v[i * 4 + 1] = u.y; v[i * 4 + 2] = u.z; v[i * 4 + 3] = u.w;
+  }
+}
+
+__device__ __forceinline__ void store_bf16x32(void* p, const float (&v)[32]) {
+  uint4* q = reinterpret_cast<uint4*>(p);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint4 u;
+    u.x = pack_bf16x2(v[i * 8 + 0], v[i * 8 + 1]);
+    u.y = pack_bf16x2(v[i * 8 + 2], v[i * 8 + 3]);
+    u.z = pack_bf16x2(v[i * 8 + 4], v[i * 8 + 5]);
+    u.w = pack_bf16x2(v[i * 8 + 6], v[i * 8 + 7]);
+    q[i] = u;
+  }
+}
+
+__device__ __forceinline__ void store_f32x32(void* p, const float (&v)[32]) {
+  float4* q = reinterpret_cast<float4*>(p);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) q[i] = make_float4(v[i * 4], v[i * 4 + 1], v[i * 4 + 2], v[i * 4 + 3]);
+}
+
+// One 32-column chunk of one accumulator row: apply the epilogue and store.
+__device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, const TileCoord& tc, int row, int n,
+                                               float (&v)[32]) {
+  switch (a.epi) {
+    case EPI_ACT_BF16: {
+      if (a.bias_g[tc.g]) {
+        float b[32];
+        load_bf16x32(static_cast<const uint16_t*>(a.bias_g[tc.g]) + n, b);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] += b[j];
+      }
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = act_apply(v[j], a.act);
+      uint16_t* o = static_cast<uint16_t*>(a.out) + static_cast<int64_t>(row) * a.ld_out +
+                    static_cast<int64_t>(tc.g) * a.out_col_per_group + n;
+      store_bf16x32(o, v);
+      break;
+    }
+    case EPI_PARTIAL_F32: {
+      float* o = static_cast<float*>(a.out) + static_cast<int64_t>(tc.g) * a.out_group_stride +
+                 static_cast<int64_t>(row) * a.ld_out + n;
+      store_f32x32(o, v);
+      break;
+    }
+    case EPI_BIAS_RESID: {
+      if (a.bias) {
+        float b[32];
+        load_bf16x32(static_cast<const uint16_t*>(a.bias) + n, b);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] += b[j];
+      }
+      if (a.resid) {
+        float r[32];
+        if (a.resid_fp32)
+          load_f32x32(static_cast<const float*>(a.resid) + static_cast<int64_t>(row) * a.ld_resid + n, r);
+        else
+          load_bf16x32(static_cast<const uint16_t*>(a.resid) + static_cast<int64_t>(row) * a.ld_resid + n, r);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] += r[j];
+      }
+      if (a.out_fp32)
+        store_f32x32(static_cast<float*>(a.out) + static_cast<int64_t>(row) * a.ld_out + n, v);
+      else
+        store_bf16x32(static_cast<uint16_t*>(a.out) + static_cast<int64_t>(row) * a.ld_out + n, v);
+      break;
+    }
+    case EPI_QKV: {
+      if (a.bias_g[tc.g]) {
+        float b[32];
+        load_bf16x32(static_cast<const uint16_t*>(a.bias_g[tc.g]) + n, b);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] += b[j];
+      }
+      const int per = a.Hg * a.d;
+      const int part = n / per;
+      const int within = n - part * per;
+      const int head = tc.g * a.Hg + within / a.d;
+      const int dd = within % a.d;
+      const int b = row / a.S;
+      const int s = row - b * a.S;
+      void* base = part == 0 ? a.q : (part == 1 ? a.k : a.v);
+      uint16_t* o = static_cast<uint16_t*>(base) +
+                    ((static_cast<int64_t>(b) * a.H + head) * a.S + s) * a.d + dd;
+      store_bf16x32(o, v);
+      break;
+    }
+    default:
+      break;
+  }
+}
+
+__global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_constant__ GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment for the 128-byte-swizzled tiles.
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* full_bar = bars;                       // [STAGES]
+  uint64_t* empty_bar = bars + STAGES;             // [STAGES]
+  uint64_t* acc_full = bars + 2 * STAGES;          // [NUM_ACC]
+  uint64_t* acc_empty = bars + 2 * STAGES + NUM_ACC;  // [NUM_ACC]
+  uint64_t* drain_bar = bars + 2 * STAGES + 2 * NUM_ACC;
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  const int m_tiles = (a.M + BM - 1) / BM;
+  const int n_tiles = (a.N + BN - 1) / BN;
+  const int num_tiles = m_tiles * n_tiles * (a.concat ? 1 : a.G);
+  const int kb_per_group = a.Kg / BK;
+  const int k_iters = a.concat ? kb_per_group * a.G : kb_per_group;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int s = 0; s < NUM_ACC; ++s) {
+      mbar_init(&acc_full[s], 1);
+      mbar_init(&acc_empty[s], EPI_THREADS);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_base_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_base_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&a.tmA);
+      for (int g = 0; g < a.G; ++g) tma_prefetch_desc(&a.tmB[g]);
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const TileCoord tc = tile_coord(a, tile, m_tiles, n_tiles);
+        const int m0 = tc.m_blk * BM;
+        const int n0 = tc.n_blk * BN;
+        for (int it = 0; it < k_iters; ++it) {
+          if (*abort_flag) { ok = false; break; }
+          if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, a.wait_limit_ns, a.status, WAIT_SITE_PRODUCER)) {
+            *abort_flag = 1; ok = false; break;
+          }
+          const int g = a.concat ? it / kb_per_group : tc.g;
+          const int kb = a.concat ? it - g * kb_per_group : it;
+          mbar_arrive_expect_tx(&full_bar[stage], STAGE_BYTES);
+          tma_load_2d(sA + stage * A_STAGE_BYTES, &a.tmA, &full_bar[stage], g * a.a_k_per_group + kb * BK, m0);
+          uint8_t* b_dst = sB + stage * B_STAGE_BYTES;
+#pragma unroll
+          for (int j = 0; j < BN / 64; ++j)
+            tma_load_2d(b_dst + j * B_BLOCK_BYTES, &a.tmB[g], &full_bar[stage], n0 + j * 64, kb * BK);
+          ++issued;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // Wait for our own copies still in flight (the last min(issued, STAGES) stages).
+      const int pending = issued < STAGES ? issued : STAGES;
+      int s = stage;
+      uint32_t ph = phase;
+      for (int i = 0; i < pending; ++i) {
+        if (--s < 0) { s = STAGES - 1; ph ^= 1u; }
+        mbar_wait_bounded(&full_bar[s], ph, a.wait_limit_ns, a.status, WAIT_SITE_PRODUCER);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      const uint32_t sA_addr = smem_u32(sA);
+      const uint32_t sB_addr = smem_u32(sB);
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait_bounded(&acc_empty[acc], acc_phase ^ 1u, a.wait_limit_ns, a.status, WAIT_SITE_MMA_ACC)) {
+          *abort_flag = 1; ok = false; break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int it = 0; it < k_iters; ++it) {
+          if (*abort_flag) { ok = false; break; }
+          if (!mbar_wait_bounded(&full_bar[stage], phase, a.wait_limit_ns, a.status, WAIT_SITE_MMA_FULL)) {
+            *abort_flag = 1; ok = false; break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = sA_addr + stage * A_STAGE_BYTES;
+          const uint32_t b_base = sB_addr + stage * B_STAGE_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            // A: K-major, advance 16 elements (32 bytes) inside the swizzle atom.
+            const uint64_t adesc = smem_desc_sw128(a_base + k * 32, 16, 1024);
+            // B: N-major, advance 16 K-rows (2048 bytes); 64-column blocks 8 KB apart.
+            const uint64_t bdesc = smem_desc_sw128(b_base + k * 16 * 128, B_BLOCK_BYTES, 1024);
+            mma_bf16_ss(d_tmem, adesc, bdesc, IDESC, (it > 0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty_bar[stage]);  // frees the smem stage once these MMAs finish
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit(&acc_full[acc]);       // accumulator ready for the epilogue
+        if (++acc == NUM_ACC) { acc = 0; acc_phase ^= 1u; }
+      }
+      // Drain: wait until every MMA issued by this thread has completed.
+      mma_commit(drain_bar);
+      mbar_wait_bounded(drain_bar, 0, a.wait_limit_ns, a.status, WAIT_SITE_MMA_ACC);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    const int sub = warp & 3;               // TMEM sub-partition this warp may access
+    const int row_in_tile = sub * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      if (*abort_flag) break;
+      // the decision is made warp-uniform: tcgen05.ld below is a warp-collective instruction
+      const bool ready = __all_sync(0xffffffffu,
+                                    mbar_wait_bounded(&acc_full[acc], acc_phase, a.wait_limit_ns, a.status,
+                                                      WAIT_SITE_EPILOGUE));
+      if (!ready) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const TileCoord tc = tile_coord(a, tile, m_tiles, n_tiles);
+      const int row = tc.m_blk * BM + row_in_tile;
+      const int n0 = tc.n_blk * BN;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        const int n = n0 + c * 32;
+        if (n >= a.N) break;  // uniform over the CTA: N is a multiple of 32
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(t_row + c * 32, r);
+        tmem_ld_wait();
+        if (row < a.M) {
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          epilogue_chunk(a, tc, row, n, v);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[acc]);
+      if (++acc == NUM_ACC) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+tp_status launch_gemm(const GemmArgs& a, cudaStream_t stream, const char* name) {
+  static int attr_set[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return TP_ERR_CUDA;
+  if (dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(tp_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+        cudaSuccess)
+      return TP_ERR_CUDA;
+    attr_set[dev] = 1;
+  }
+  const int m_tiles = (a.M + BM - 1) / BM;
+  const int n_tiles = (a.N + BN - 1) / BN;
+  const long long tiles = 1LL * m_tiles * n_tiles * (a.concat ? 1 : a.G);
+  if (tiles <= 0) return TP_OK;
+  const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
+  trace_before(stream);
+  tp_gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
+  trace_after(stream, name);
+  return TP_OK;
+}
+
+}  // namespace tpb

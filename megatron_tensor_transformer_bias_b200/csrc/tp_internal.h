@@ -1,0 +1,97 @@
+// Internal launch interface between the C-ABI layer (tp_api.cu) and the kernels.
+// Host-only types; nothing here is part of the public ABI.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+#include <cstddef>
+
+#include "../../include/tpblock.h"
+
+namespace tpb {
+
+// Device status word codes (the low byte; the next byte says where a wait gave up).
+enum : uint32_t { DEV_OK = 0, DEV_TIMEOUT = 5 };
+enum : uint32_t {
+  WAIT_SITE_PRODUCER = 1, WAIT_SITE_MMA_FULL = 2, WAIT_SITE_MMA_ACC = 3,
+  WAIT_SITE_EPILOGUE = 4, WAIT_SITE_SELFTEST = 5, WAIT_SITE_ATTN = 6
+};
+
+// GEMM tile shape of the tcgen05 kernel (one CTA per SM, persistent).
+constexpr int GEMM_BM = 128;
+constexpr int GEMM_BN = 256;
+constexpr int GEMM_BK = 64;
+
+enum GemmEpilogue : int {
+  EPI_ACT_BF16 = 0,    // out[:, g*ncol + n] = act(acc + bias_g[n]) as bf16   (column-parallel layer)
+  EPI_PARTIAL_F32 = 1, // P[g][m, n] = acc as fp32                              (row layer, partials)
+  EPI_BIAS_RESID = 2,  // out[m, n] = acc + bias[n] + resid[m, n]              (row layer, fused reduce)
+  EPI_QKV = 3,         // scatter acc (+ bias_g) to Q/K/V [B, H, S, d] bf16     (QKV column layer)
+};
+
+enum Activation : int { ACT_NONE = 0, ACT_GELU = 1, ACT_RELU = 2 };
+
+struct __align__(64) GemmArgs {
+  CUtensorMap tmA;                      // A [M, Ktot] bf16 K-major, box {64, 128}, 128B swizzle
+  CUtensorMap tmB[TP_MAX_SHARDS];       // B_g [Kg, N] bf16 N-major, box {64, 64}, 128B swizzle
+  int M, N, Kg, G;
+  int concat;                           // 1: one tile sums all G K-slices in order g = 0..G-1
+  int a_k_per_group;                    // column offset of group g's K-slice in A (elements)
+  int epi, act;
+  void* out;
+  int64_t ld_out;                       // elements
+  int64_t out_col_per_group;            // EPI_ACT_BF16: column offset of group g in out
+  int64_t out_group_stride;             // EPI_PARTIAL_F32: elements between partials
+  int out_fp32;
+  const void* bias_g[TP_MAX_SHARDS];    // bf16 [N] per group, or null
+  const void* bias;                     // bf16 [N] or null (EPI_BIAS_RESID)
+  const void* resid;                    // [M, N] or null
+  int64_t ld_resid;
+  int resid_fp32;
+  // EPI_QKV scatter: column c of group g -> part c / (Hg*d), head g*Hg + (c % (Hg*d)) / d
+  void* q; void* k; void* v;
+  int S, H, Hg, d;
+  uint32_t* status;
+  uint64_t wait_limit_ns;
+};
+
+struct AttnArgs {
+  CUtensorMap tmQ;   // Q [B*H*S, d] bf16, box {64, 128}, 128B swizzle
+  CUtensorMap tmK;   // K [B*H*S, d]
+  CUtensorMap tmV;   // V [B*H*S, d]
+  void* O;           // O [B*S, H*d] bf16 (head-major columns)
+  int B, S, H, d, causal;
+  int head0;         // first head handled (head-group offset)
+  float scale_log2;  // log2(e) / sqrt(d)
+  uint32_t* status;
+  uint64_t wait_limit_ns;
+};
+
+// Per-device runtime facts.
+int sm_count();
+uint32_t* device_status_ptr();
+uint64_t wait_limit_ns();
+
+// Tensor-map construction (driver entry point fetched through the runtime).
+tp_status make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                            uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+
+// Kernel launchers.  All are asynchronous on `stream` and validate nothing:
+// the C-ABI layer has checked every argument before calling them.
+tp_status launch_gemm(const GemmArgs& a, cudaStream_t stream, const char* name);
+tp_status launch_attention(const AttnArgs& a, cudaStream_t stream);
+tp_status launch_reduce_partials(const float* P, int t, int64_t M, int64_t h, const void* bias, int bias_fp32,
+                                 const void* resid, int resid_fp32, void* out, int out_fp32,
+                                 cudaStream_t stream);
+tp_status launch_layernorm(const void* x, int in_fp32, const void* g, const void* b, int64_t M, int64_t h,
+                           float eps, void* y, cudaStream_t stream);
+tp_status launch_ffn_fp32(const float* X, int64_t M, int64_t h, int64_t f, int t, const tp_shard* W1,
+                          const void* const* b1, const tp_shard* W2, const float* b2, const float* resid,
+                          float* out, int act, float* Z, float* P, cudaStream_t stream);
+tp_status launch_selftest_wait(uint64_t limit_ns, cudaStream_t stream);
+
+// Launch tracing (tp_trace_*): brackets each kernel launch with events.
+void trace_before(cudaStream_t stream);
+void trace_after(cudaStream_t stream, const char* name);
+
+}  // namespace tpb

@@ -1,0 +1,129 @@
+"""GPU parity of the attention sub-layer and the pre-LN layer against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from megatron_tensor_transformer_bias_b200 import configs, inputs
+from megatron_tensor_transformer_bias_b200 import tpblock as tb
+from tests.parity import assert_bf16_close, to64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _attn_gpu(a, B, S, H, d, t, causal=True, mode="fused", perm=None, with_bo=True, with_res=True):
+    Wqkv = inputs.pack_qkv(a["Wq"], a["Wk"], a["Wv"], t, H, d)
+    shards = tb.shard_columns(Wqkv, t)
+    Wo = tb.shard_rows(a["Wo"], t)
+    if perm is not None:
+        shards = [shards[i] for i in perm]
+        Wo = [Wo[i] for i in perm]
+    out = torch.empty_like(a["X"])
+    tb.tp_attn_forward(a["X"], B, S, H, d, shards, None, Wo, a["bo"] if with_bo else None,
+                       a["X"] if with_res else None, out, causal=causal, mode=mode)
+    assert tb.tp_get_device_status() == tb.TP_OK
+    return out
+
+
+def _attn_ref(a, B, S, H, d, causal=True, rows=None, with_bo=True, with_res=True):
+    return oracle.attn_forward(to64(a["X"]), to64(a["Wq"]), to64(a["Wk"]), to64(a["Wv"]), to64(a["Wo"]),
+                               to64(a["bo"]) if with_bo else None, to64(a["X"]) if with_res else None,
+                               B, S, H, d, causal=causal, rows=rows)
+
+
+SMALL = [(2, 200, 256, 4), (1, 128, 256, 2), (1, 1, 128, 1), (3, 129, 512, 4), (1, 384, 256, 2)]
+
+
+@pytest.mark.parametrize("B,S,h,H", SMALL)
+@pytest.mark.parametrize("causal", [True, False])
+def test_attention_small_full(B, S, h, H, causal):
+    d = 128
+    a = inputs.attn_inputs(B, S, h, H, d, seed=11, device=DEV)
+    ref = _attn_ref(a, B, S, H, d, causal)
+    for t in sorted({1, H // 2 if H >= 2 else 1, H}):
+        if H % t:
+            continue
+        out = _attn_gpu(a, B, S, H, d, t, causal)
+        assert_bf16_close(out, ref, f"B{B} S{S} h{h} H{H} t{t} causal={causal}")
+
+
+def test_attention_partials_mode_and_head_permutation():
+    B, S, h, H, d = 2, 256, 512, 4, 128
+    a = inputs.attn_inputs(B, S, h, H, d, seed=12, device=DEV)
+    ref = _attn_ref(a, B, S, H, d)
+    assert_bf16_close(_attn_gpu(a, B, S, H, d, 4, mode="partials"), ref, "partials")
+    # permuting head groups across shards (with their Wo rows) leaves the output unchanged
+    assert_bf16_close(_attn_gpu(a, B, S, H, d, 4, perm=[2, 0, 3, 1]), ref, "permuted groups")
+
+
+def test_attention_first_token_closed_form():
+    """Causal row 0 of each sequence attends only to itself: out = X0 Wv Wo + bo + X0."""
+    B, S, h, H, d = 2, 160, 256, 2, 128
+    a = inputs.attn_inputs(B, S, h, H, d, seed=13, device=DEV)
+    out = _attn_gpu(a, B, S, H, d, 2)
+    for b in range(B):
+        r = b * S
+        x0 = to64(a["X"][r])
+        want = x0 @ to64(a["Wv"]) @ to64(a["Wo"]) + to64(a["bo"]) + x0
+        assert_bf16_close(out[r:r + 1], want[None], f"first token of sequence {b}")
+
+
+@pytest.fixture(scope="module")
+def attn_full():
+    w = configs.ATTN_B2_S2048
+    a = inputs.attn_inputs(w.B, w.S, w.h, w.H, w.d, seed=0, device=DEV)
+    rows = inputs.sample_rows(w.M, configs.SAMPLED_ROWS, seq=w.S)
+    ref = _attn_ref(a, w.B, w.S, w.H, w.d, True, rows=rows)
+    yield w, a, rows, ref
+    del a
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("mode", ["fused", "partials"])
+def test_attention_B2_S2048_sampled(attn_full, mode):
+    w, a, rows, ref = attn_full
+    out = _attn_gpu(a, w.B, w.S, w.H, w.d, w.t, True, mode=mode)
+    assert_bf16_close(out[rows], ref, f"attention B2 S2048 t4 {mode}")
+    assert torch.isfinite(out.float()).all()
+
+
+# ---------------------------------------------------------------- layer
+def _layer_gpu(p, B, S, H, d, t, causal=True, mode="fused"):
+    Wqkv = tb.shard_columns(inputs.pack_qkv(p["Wq"], p["Wk"], p["Wv"], t, H, d), t)
+    out = torch.empty_like(p["X"])
+    tb.tp_layer_forward(p["X"], B, S, H, d, p["ln1_g"], p["ln1_b"], Wqkv, None, tb.shard_rows(p["Wo"], t),
+                        p["bo"], p["ln2_g"], p["ln2_b"], tb.shard_columns(p["W1"], t),
+                        tb.shard_vector(p["b1"], t), tb.shard_rows(p["W2"], t), p["b2"], out, eps=1e-5,
+                        causal=causal, mode=mode)
+    assert tb.tp_get_device_status() == tb.TP_OK
+    return out
+
+
+def _layer_ref(p, B, S, H, d, causal=True, rows=None):
+    q = {k: to64(v) for k, v in p.items()}
+    return oracle.layer_forward(q["X"], q, B, S, H, d, eps=1e-5, causal=causal, rows=rows)
+
+
+@pytest.mark.parametrize("mode", ["fused", "partials"])
+@pytest.mark.parametrize("causal", [True, False])
+def test_layer_small_full(mode, causal):
+    B, S, h, H, d, f, t = 2, 150, 256, 4, 128, 1024, 2
+    p = inputs.layer_inputs(B, S, h, H, d, f, seed=14, device=DEV)
+    g = torch.Generator(device=DEV).manual_seed(15)
+    p["ln1_g"] = (1 + 0.1 * torch.randn(h, generator=g, device=DEV)).to(torch.bfloat16)
+    p["ln1_b"] = (0.1 * torch.randn(h, generator=g, device=DEV)).to(torch.bfloat16)
+    out = _layer_gpu(p, B, S, H, d, t, causal, mode)
+    assert_bf16_close(out, _layer_ref(p, B, S, H, d, causal), f"layer {mode} causal={causal}")
+
+
+def test_layer_S2048_h8192_sampled():
+    w = configs.LAYER_S2048_H8192
+    p = inputs.layer_inputs(w.B, w.S, w.h, w.H, w.d, w.f, seed=0, device=DEV)
+    rows = inputs.sample_rows(w.M, configs.SAMPLED_ROWS, seq=w.S)
+    ref = _layer_ref(p, w.B, w.S, w.H, w.d, True, rows=rows)
+    out = _layer_gpu(p, w.B, w.S, w.H, w.d, w.t)
+    assert_bf16_close(out[rows], ref, "layer B1 S2048 h8192 t8")
+    assert torch.isfinite(out.float()).all()
+    del p
+    torch.cuda.empty_cache()

@@ -1,0 +1,179 @@
+"""GPU parity of the FFN block and the parallel linears against the fp64 oracle.
+
+Small cases compare every element; full-size workloads compare a seeded sample
+of 64 token rows.  All calls go through the C-ABI (ctypes binding)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from megatron_tensor_transformer_bias_b200 import configs, inputs
+from megatron_tensor_transformer_bias_b200 import tpblock as tb
+from tests.parity import assert_bf16_close, assert_fp32_close, ffn_oracle_rows, to64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _run_ffn(inp, t, mode="fused", act="gelu", with_b1=True, with_b2=True, with_res=True):
+    X = inp["X"]
+    W1s = tb.shard_columns(inp["W1"], t)
+    W2s = tb.shard_rows(inp["W2"], t)
+    b1s = tb.shard_vector(inp["b1"], t) if with_b1 else None
+    out = torch.empty_like(X)
+    tb.tp_ffn_forward(X, W1s, b1s, W2s, inp["b2"] if with_b2 else None, X if with_res else None, out,
+                      mode=mode, act=act)
+    assert tb.tp_get_device_status() == tb.TP_OK
+    return out
+
+
+def _oracle_full(inp, act="gelu", with_b1=True, with_b2=True, with_res=True):
+    X = to64(inp["X"])
+    return oracle.ffn_forward(X, to64(inp["W1"]), to64(inp["b1"]) if with_b1 else None, to64(inp["W2"]),
+                              to64(inp["b2"]) if with_b2 else None, X if with_res else None, act=act)
+
+
+# ---------------------------------------------------------------- tiny fp32 workload
+def test_fp32_tiny_workload_full():
+    w = configs.TINY_FP32_FFN
+    inp = inputs.ffn_inputs(w.M, w.h, w.f, "fp32", seed=0, device=DEV)
+    out = _run_ffn(inp, w.t)
+    assert out.dtype == torch.float32
+    assert_fp32_close(out, _oracle_full(inp), "fp32 M8 h64 f256 t2")
+
+
+@pytest.mark.parametrize("t", [1, 2, 4, 8])
+def test_fp32_sharding_invariance(t):
+    inp = inputs.ffn_inputs(8, 64, 256, "fp32", seed=0, device=DEV)
+    assert_fp32_close(_run_ffn(inp, t), _oracle_full(inp), f"fp32 t={t}")
+
+
+# ---------------------------------------------------------------- small bf16 cases (every element)
+SMALL = [(300, 256, 1024), (128, 128, 512), (1, 64, 256), (513, 512, 2048)]
+
+
+@pytest.mark.parametrize("M,h,f", SMALL)
+@pytest.mark.parametrize("t", [1, 2, 4])
+@pytest.mark.parametrize("mode", ["fused", "partials"])
+def test_bf16_small_full(M, h, f, t, mode):
+    inp = inputs.ffn_inputs(M, h, f, "bf16", seed=1, device=DEV)
+    out = _run_ffn(inp, t, mode=mode)
+    assert_bf16_close(out, _oracle_full(inp), f"M{M} h{h} f{f} t{t} {mode}")
+
+
+def test_bf16_relu_and_no_bias():
+    inp = inputs.ffn_inputs(200, 256, 1024, "bf16", seed=2, device=DEV)
+    out = _run_ffn(inp, 2, act="relu")
+    assert_bf16_close(out, _oracle_full(inp, act="relu"), "relu")
+    out = _run_ffn(inp, 4, with_b1=False, with_b2=False, with_res=False)
+    assert_bf16_close(out, _oracle_full(inp, with_b1=False, with_b2=False, with_res=False), "no bias/residual")
+
+
+def test_bf16_sharding_invariance_bitwise_and_determinism():
+    """Fused mode sums the shards' K-slices in one accumulator in the same order
+    for every t, so the output is the same bits for every t dividing f/64."""
+    inp = inputs.ffn_inputs(384, 256, 2048, "bf16", seed=3, device=DEV)
+    ref = _run_ffn(inp, 1)
+    for t in (2, 4, 8):
+        assert torch.equal(_run_ffn(inp, t), ref), f"t={t} differs from t=1"
+    for mode in ("fused", "partials"):
+        a = _run_ffn(inp, 4, mode=mode)
+        b = _run_ffn(inp, 4, mode=mode)
+        assert torch.equal(a, b), f"{mode} not deterministic"
+
+
+def test_bf16_special_cases():
+    inp = inputs.ffn_inputs(130, 128, 512, "bf16", seed=4, device=DEV)
+    # W2 = 0: out = b2 + residual
+    z = dict(inp)
+    z["W2"] = torch.zeros_like(inp["W2"])
+    out = _run_ffn(z, 2)
+    want = (inp["X"].float() + inp["b2"].float()).to(torch.bfloat16)
+    assert torch.equal(out, want)
+    # X = 0 (no residual): out = GeLU(b1) W2 + b2
+    z = dict(inp)
+    z["X"] = torch.zeros_like(inp["X"])
+    out = _run_ffn(z, 4, with_res=False)
+    assert_bf16_close(out, _oracle_full(z, with_res=False), "X=0")
+
+
+def test_shards_in_separate_buffers():
+    """Shards need not be views of one matrix: copy each into its own buffer."""
+    inp = inputs.ffn_inputs(256, 256, 1024, "bf16", seed=5, device=DEV)
+    t = 4
+    W1s = [w.contiguous() for w in tb.shard_columns(inp["W1"], t)]
+    W2s = [w.clone() for w in tb.shard_rows(inp["W2"], t)]
+    b1s = [b.clone() for b in tb.shard_vector(inp["b1"], t)]
+    out = torch.empty_like(inp["X"])
+    tb.tp_ffn_forward(inp["X"], W1s, b1s, W2s, inp["b2"], inp["X"], out)
+    assert_bf16_close(out, _oracle_full(inp), "separate shard buffers")
+
+
+# ---------------------------------------------------------------- parallel linears alone
+@pytest.mark.parametrize("act", [None, "gelu", "relu"])
+def test_column_linear(act):
+    M, k, n, t = 200, 256, 1024, 4
+    inp = inputs.ffn_inputs(M, k, n, "bf16", seed=6, device=DEV)
+    out = torch.empty(M, n, dtype=torch.bfloat16, device=DEV)
+    tb.tp_column_linear_forward(inp["X"], tb.shard_columns(inp["W1"], t), tb.shard_vector(inp["b1"], t), out,
+                                act=act)
+    Z = to64(inp["X"]) @ to64(inp["W1"]) + to64(inp["b1"])
+    ref = {None: Z, "gelu": oracle.gelu(Z) if act == "gelu" else None, "relu": oracle.relu(Z)}[act]
+    assert_bf16_close(out, ref, f"column linear {act}")
+
+
+@pytest.mark.parametrize("mode", ["fused", "partials"])
+def test_row_linear(mode):
+    M, k, n, t = 300, 1024, 256, 4
+    g = torch.Generator(device=DEV).manual_seed(7)
+    A = torch.randn(M, k, generator=g, device=DEV).to(torch.bfloat16)
+    W = (torch.randn(k, n, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    bias = (torch.randn(n, generator=g, device=DEV) * 0.01).to(torch.bfloat16)
+    R = torch.randn(M, n, generator=g, device=DEV).to(torch.bfloat16)
+    out = torch.empty(M, n, dtype=torch.bfloat16, device=DEV)
+    tb.tp_row_linear_forward(A, tb.shard_rows(W, t), bias, R, out, mode=mode)
+    ref = oracle.reduce_partials([to64(A[:, i * k // t:(i + 1) * k // t]) @ to64(W[i * k // t:(i + 1) * k // t])
+                                  for i in range(t)], to64(bias), to64(R))
+    assert_bf16_close(out, ref, f"row linear {mode}")
+
+
+# ---------------------------------------------------------------- full-size workloads (sampled rows)
+@pytest.fixture(scope="module")
+def ffn_2048():
+    w = configs.ffn_2048x4096x16384(4)
+    inp = inputs.ffn_inputs(w.M, w.h, w.f, "bf16", seed=0, device=DEV)
+    rows = inputs.sample_rows(w.M, configs.SAMPLED_ROWS, seq=w.seq)
+    ref = ffn_oracle_rows(inp, rows)
+    yield inp, rows, ref
+    del inp
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("t", configs.FFN_SHARD_COUNTS)
+@pytest.mark.parametrize("mode", ["fused", "partials"])
+def test_ffn_2048x4096x16384_sampled(ffn_2048, t, mode):
+    inp, rows, ref = ffn_2048
+    out = _run_ffn(inp, t, mode=mode)
+    assert_bf16_close(out[rows], ref, f"M2048 h4096 f16384 t{t} {mode}")
+    # properties that hold at every row: finite, and fused output bit-identical across t
+    assert torch.isfinite(out.float()).all()
+
+
+def test_ffn_2048_bitwise_across_t(ffn_2048):
+    inp, _, _ = ffn_2048
+    ref = _run_ffn(inp, 1)
+    for t in (2, 4, 8):
+        assert torch.equal(_run_ffn(inp, t), ref)
+
+
+@pytest.mark.parametrize("h", configs.SWEEP_HIDDEN)
+def test_ffn_hidden_sweep_sampled(h):
+    M = 4096
+    inp = inputs.ffn_inputs(M, h, 4 * h, "bf16", seed=0, device=DEV)
+    rows = inputs.sample_rows(M, configs.SAMPLED_ROWS)
+    ref = ffn_oracle_rows(inp, rows, chunks=16)
+    for t in configs.SWEEP_SHARDS:
+        out = _run_ffn(inp, t)
+        assert_bf16_close(out[rows], ref, f"M4096 h{h} t{t}")
+    del inp, out
+    torch.cuda.empty_cache()
