@@ -65,7 +65,7 @@ typedef enum {
   TP_ERR_TIMEOUT = 5      /* a device wait ran out (reported by tp_get_device_status) */
 } tp_status;
 
-typedef enum { TP_BF16 = 0, TP_FP32 = 1 } tp_dtype;
+typedef enum { TP_BF16 = 0, TP_FP32 = 1, TP_FP16 = 2 } tp_dtype;
 
 /* How step 3 (the all-reduce) is done on one device.
  * TP_REDUCE_FUSED:    one row-GEMM tile accumulates the K-slices of all t
@@ -79,9 +79,17 @@ typedef enum { TP_REDUCE_FUSED = 0, TP_REDUCE_PARTIALS = 1 } tp_reduce_mode;
 /* Element-wise nonlinearity of step 1: exact GeLU z*Phi(z) (erf form) or ReLU. */
 typedef enum { TP_ACT_GELU = 0, TP_ACT_RELU = 1 } tp_activation;
 
+/* A weight shard.  `dtype` is TP_BF16 (0, so a zeroed struct means bf16) or
+ * TP_FP16; every shard of one weight has the same dtype.  In each tensor-core
+ * GEMM the activation operand is produced in its weight's type: an fp16 W2
+ * makes act(Z) fp16, an fp16 Wqkv makes the layer's LN1 output fp16, and so on.
+ * fp16 has 3 more mantissa bits than bf16 at the same tensor-core rate, and
+ * bf16 weights of ordinary magnitude convert to fp16 exactly. */
 typedef struct {
   const void* ptr; /* device pointer to element (0, 0) of the shard */
   int64_t ld;      /* row stride in elements */
+  int32_t dtype;   /* TP_BF16 or TP_FP16 */
+  int32_t reserved;
 } tp_shard;
 
 typedef void* tp_stream_t; /* cudaStream_t */
@@ -90,9 +98,10 @@ typedef void* tp_stream_t; /* cudaStream_t */
  * [TP-CR] steps 1-3:  out = sum_{i<t} act(X W1_i + b1_i) W2_i + b2 + residual.
  *
  *  X        [M, h], dtype, ld = h (contiguous).
- *  W1[i]    [h, f/t] view, i < t (column shard i of W1 [h, f]).
+ *  W1[i]    [h, f/t] view, i < t (column shard i of W1 [h, f]); same dtype as X.
  *  b1       array of t pointers to [f/t] vectors, or NULL (no bias).
- *  W2[i]    [f/t, h] view (row shard i of W2 [f, h]).
+ *  W2[i]    [f/t, h] view (row shard i of W2 [f, h]); TP_BF16 or TP_FP16
+ *           (act(Z) is stored in the same type).
  *  b2       [h] or NULL; added once, after the sum over shards.
  *  residual [M, h] or NULL; added after the sum (may alias X).
  *  out      [M, h], contiguous; must not alias X, residual or the weights.
@@ -118,10 +127,11 @@ TP_API tp_status tp_ffn_forward_act(const void* X, int64_t M, int64_t h, int64_t
                              size_t ws_bytes, tp_stream_t stream);
 
 /* ------------------------------------------------------------------ parallel linears
- * Column-parallel linear alone ([TP-CR] step 1), bf16:
+ * Column-parallel linear alone ([TP-CR] step 1), bf16 or fp16 (W's dtype):
  *   out[:, i*n/t : (i+1)*n/t] = act(X W_i + b_i)   for i < t,
- *   X [M, k] contiguous, W[i] [k, n/t] views, b NULL or t pointers to [n/t],
- *   out [M, n] contiguous bf16.  act: -1 = identity, else tp_activation. */
+ *   X [M, k] contiguous, W[i] [k, n/t] views, b NULL or t pointers to [n/t] bf16,
+ *   out [M, n] contiguous.  X and out have W's dtype.
+ *   act: -1 = identity, else tp_activation. */
 TP_API tp_status tp_column_linear_forward(const void* X, int64_t M, int64_t k, int64_t n, int t, const tp_shard* W,
                                    const void* const* b, int act, void* out, tp_stream_t stream);
 
@@ -144,10 +154,14 @@ TP_API tp_status tp_row_linear_forward(const void* A, int64_t M, int64_t k, int6
  *   O_i = concat over heads g of group i of softmax(Q_g K_g^T / sqrt(d) + mask) V_g.
  *
  *  X        [B*S, h] bf16 contiguous (row r = b*S + s).
- *  Wqkv[i]  [h, 3*Hg*d] view, Hg = heads/t: columns [Q heads | K heads | V heads]
+ *  Wqkv[i]  [h, 3*Hg*d] bf16 view, Hg = heads/t: columns [Q heads | K heads | V heads]
  *           of group i, head g of the group at columns g*d .. g*d+d-1 of each block.
+ *           Q, K, V, the softmax weights P and the tensor-core operands of
+ *           Q K^T and P V are fp16 (the scores' sensitivity to rounding of Q and
+ *           K grows with their magnitude); accumulation is fp32.
  *  bqkv     NULL or t pointers to [3*Hg*d] bf16.
- *  Wo[i]    [Hg*d, h] view (rows of the output projection for group i's heads).
+ *  Wo[i]    [Hg*d, h] view (rows of the output projection for group i's heads),
+ *           TP_BF16 or TP_FP16 (the attention output O is stored in that type).
  *  bo       [h] or NULL.  residual [B*S, h] or NULL.  out [B*S, h] bf16.
  *  causal   1: key j is visible to query i iff j <= i (same sequence); 0: all keys.
  * Limits: d == 128, heads % t == 0, S >= 1.
@@ -163,7 +177,9 @@ TP_API tp_status tp_attn_forward(const void* X, int B, int S, int h, int heads, 
  *   h1  = X + Attn(LN1(X))            (h1 kept in fp32 inside the workspace)
  *   out = h1 + FFN(LN2(h1))           (bf16)
  * LayerNorm runs replicated over the full row ([TP-CR], feature reductions).
- * Weights as in tp_attn_forward and tp_ffn_forward; ln*_g / ln*_b are [h] bf16.
+ * Weights as in tp_attn_forward and tp_ffn_forward, except that every weight
+ * may be TP_BF16 or TP_FP16: LN1's output takes Wqkv's type, O takes Wo's, LN2's
+ * output takes W1's and act(Z) takes W2's.  ln*_g / ln*_b are [h] bf16.
  */
 TP_API size_t tp_layer_workspace_bytes(int B, int S, int h, int heads, int d, int64_t f, int t, tp_reduce_mode mode);
 TP_API tp_status tp_layer_forward(const void* X, int B, int S, int h, int heads, int d, int64_t f, int t,
@@ -176,9 +192,9 @@ TP_API tp_status tp_layer_forward(const void* X, int B, int S, int h, int heads,
 /* ------------------------------------------------------------------ building blocks
  * LayerNorm over rows: y = (x - mean) / sqrt(var + eps) * gamma + beta, var the
  * biased variance.  x [M, h] bf16 or fp32 (in_dtype); gamma, beta [h] bf16 or
- * NULL (1 and 0); y [M, h] bf16.  h % 8 == 0. */
+ * NULL (1 and 0); y [M, h] in out_dtype (TP_BF16 or TP_FP16).  h % 8 == 0. */
 TP_API tp_status tp_layernorm_forward(const void* x, tp_dtype in_dtype, const void* gamma, const void* beta, int64_t M,
-                               int64_t h, float eps, void* y, tp_stream_t stream);
+                               int64_t h, float eps, void* y, tp_dtype out_dtype, tp_stream_t stream);
 
 /* Step 3 alone: out = sum_{i<t} P[i] + bias + residual in fixed order i = 0..t-1.
  * P [t, M, h] fp32 contiguous; bias [h] and residual [M, h] in `dtype` or NULL;

@@ -118,22 +118,23 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-tp_status make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                            uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+tp_status make_tmap_2d(CUtensorMap* map, const void* base, int f16, uint64_t inner, uint64_t outer,
+                       uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_stride_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return TP_OK;
 }
 
-static tp_status make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+static tp_status make_tmap_f16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                                    uint64_t s1_bytes, uint64_t s2_bytes, uint32_t b0, uint32_t b1) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
@@ -141,7 +142,7 @@ static tp_status make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t 
   cuuint64_t strides[2] = {s1_bytes, s2_bytes};
   cuuint32_t box[3] = {b0, b1, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled(3d) failed (%d)", static_cast<int>(r));
@@ -149,8 +150,8 @@ static tp_status make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t 
 }
 
 tp_status make_tmap_attn(CUtensorMap* map, const void* base, int BH, int S, int d) {
-  // [B*H][S][d] bf16: inner d (box 64), then S (box 128), then heads (box 1).
-  return make_tmap_bf16_3d(map, base, static_cast<uint64_t>(d), static_cast<uint64_t>(S),
+  // [B*H][S][d] fp16: inner d (box 64), then S (box 128), then heads (box 1).
+  return make_tmap_f16_3d(map, base, static_cast<uint64_t>(d), static_cast<uint64_t>(S),
                            static_cast<uint64_t>(BH), static_cast<uint64_t>(d) * 2,
                            static_cast<uint64_t>(S) * d * 2, 64, 128);
 }
@@ -175,6 +176,9 @@ tp_status check_ptr(const void* p, const char* what, bool need) {
 tp_status check_shards(const tp_shard* W, int t, int64_t cols, const char* what) {
   if (!W) return fail(TP_ERR_INVALID_ARG, "%s shard array is NULL", what);
   for (int i = 0; i < t; ++i) {
+    if (W[i].dtype != TP_BF16 && W[i].dtype != TP_FP16)
+      return fail(TP_ERR_INVALID_ARG, "%s[%d].dtype=%d (weights are TP_BF16 or TP_FP16)", what, i, W[i].dtype);
+    if (W[i].dtype != W[0].dtype) return fail(TP_ERR_INVALID_ARG, "%s shards mix dtypes", what);
     if (!W[i].ptr) return fail(TP_ERR_INVALID_ARG, "%s[%d].ptr is NULL", what, i);
     if (!aligned16(W[i].ptr)) return fail(TP_ERR_INVALID_ARG, "%s[%d].ptr is not 16-byte aligned", what, i);
     if (W[i].ld < cols) return fail(TP_ERR_INVALID_ARG, "%s[%d].ld=%lld < %lld columns", what, i,
@@ -191,6 +195,8 @@ tp_status check_bias_array(const void* const* b, int t, const char* what) {
     if (b[i] && !aligned16(b[i])) return fail(TP_ERR_INVALID_ARG, "%s[%d] is not 16-byte aligned", what, i);
   return TP_OK;
 }
+
+inline int is_f16(const tp_shard* W) { return W[0].dtype == TP_FP16 ? 1 : 0; }
 
 #define TP_TRY(expr)                   \
   do {                                 \
@@ -218,36 +224,41 @@ tp_status validate_ffn_bf16_dims(int64_t M, int64_t h, int64_t f, int t) {
 }
 
 // Column-parallel GEMM: out[:, g*ncol + n] = act(X W_g + b_g), X [M, k].
+// X has W's dtype; out is written in out_type.
 tp_status run_column(const void* X, int64_t M, int64_t k, int64_t ncol, int t, const tp_shard* W,
-                     const void* const* b, int act, void* out, int64_t ld_out, cudaStream_t stream) {
+                     const void* const* b, int act, void* out, int out_type, int64_t ld_out, cudaStream_t stream) {
   GemmArgs a;
   memset(&a, 0, sizeof(a));
-  TP_TRY(make_tmap_bf16_2d(&a.tmA, X, k, M, k * 2, 64, GEMM_BM));
-  for (int i = 0; i < t; ++i) TP_TRY(make_tmap_bf16_2d(&a.tmB[i], W[i].ptr, ncol, k, W[i].ld * 2, 64, 64));
+  const int f16 = is_f16(W);
+  TP_TRY(make_tmap_2d(&a.tmA, X, f16, k, M, k * 2, 64, GEMM_BM));
+  for (int i = 0; i < t; ++i) TP_TRY(make_tmap_2d(&a.tmB[i], W[i].ptr, f16, ncol, k, W[i].ld * 2, 64, 64));
   a.M = static_cast<int>(M); a.N = static_cast<int>(ncol); a.Kg = static_cast<int>(k); a.G = t;
   a.concat = 0; a.a_k_per_group = 0;
-  a.epi = EPI_ACT_BF16; a.act = act;
-  a.out = out; a.ld_out = ld_out; a.out_col_per_group = ncol;
+  a.epi = EPI_ACT; a.act = act; a.ab_f16 = f16;
+  a.out = out; a.ld_out = ld_out; a.out_col_per_group = ncol; a.out_type = out_type;
   for (int i = 0; i < t; ++i) a.bias_g[i] = b ? b[i] : nullptr;
   a.status = device_status_ptr(); a.wait_limit_ns = wait_limit_ns();
   return launch_gemm(a, stream, "gemm_column_act");
 }
 
 // Row-parallel GEMM + reduction: out = sum_g A[:, g*kg:(g+1)*kg] W_g + bias + resid.
+// A has W's dtype; out is bf16 or fp32 (out_fp32).
 tp_status run_row(const void* A, int64_t M, int64_t kg, int64_t n, int t, const tp_shard* W, const void* bias,
                   const void* resid, int resid_fp32, void* out, int out_fp32, tp_reduce_mode mode, float* P,
                   cudaStream_t stream) {
   GemmArgs a;
   memset(&a, 0, sizeof(a));
-  TP_TRY(make_tmap_bf16_2d(&a.tmA, A, kg * t, M, kg * t * 2, 64, GEMM_BM));
-  for (int i = 0; i < t; ++i) TP_TRY(make_tmap_bf16_2d(&a.tmB[i], W[i].ptr, n, kg, W[i].ld * 2, 64, 64));
+  const int f16 = is_f16(W);
+  TP_TRY(make_tmap_2d(&a.tmA, A, f16, kg * t, M, kg * t * 2, 64, GEMM_BM));
+  for (int i = 0; i < t; ++i) TP_TRY(make_tmap_2d(&a.tmB[i], W[i].ptr, f16, n, kg, W[i].ld * 2, 64, 64));
+  a.ab_f16 = f16;
   a.M = static_cast<int>(M); a.N = static_cast<int>(n); a.Kg = static_cast<int>(kg); a.G = t;
   a.a_k_per_group = static_cast<int>(kg);
   a.status = device_status_ptr(); a.wait_limit_ns = wait_limit_ns();
   if (mode == TP_REDUCE_FUSED) {
     a.concat = 1;
     a.epi = EPI_BIAS_RESID;
-    a.out = out; a.ld_out = n; a.out_fp32 = out_fp32;
+    a.out = out; a.ld_out = n; a.out_type = out_fp32 ? OUT_F32 : OUT_BF16;
     a.bias = bias; a.resid = resid; a.ld_resid = n; a.resid_fp32 = resid_fp32;
     return launch_gemm(a, stream, "gemm_row_fused_reduce");
   }
@@ -258,6 +269,7 @@ tp_status run_row(const void* A, int64_t M, int64_t kg, int64_t n, int t, const 
   return launch_reduce_partials(P, t, M, n, bias, 0, resid, resid_fp32, out, out_fp32, stream);
 }
 
+// X has W1's dtype; act(Z) is stored in W2's dtype.
 tp_status ffn_bf16(const void* X, int64_t M, int64_t h, int64_t f, int t, const tp_shard* W1,
                    const void* const* b1, const tp_shard* W2, const void* b2, const void* resid, int resid_fp32,
                    void* out, int out_fp32, tp_reduce_mode mode, int act, void* ws, cudaStream_t stream) {
@@ -265,7 +277,7 @@ tp_status ffn_bf16(const void* X, int64_t M, int64_t h, int64_t f, int t, const 
   const int64_t fs = f / t;
   uint16_t* Zh = static_cast<uint16_t*>(ws);
   float* P = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align_up(static_cast<size_t>(M) * f * 2));
-  TP_TRY(run_column(X, M, h, fs, t, W1, b1, act, Zh, f, stream));
+  TP_TRY(run_column(X, M, h, fs, t, W1, b1, act, Zh, is_f16(W2) ? OUT_F16 : OUT_BF16, f, stream));
   return run_row(Zh, M, fs, h, t, W2, b2, resid, resid_fp32, out, out_fp32, mode, P, stream);
 }
 
@@ -293,6 +305,9 @@ tp_status validate_ffn(const void* X, int64_t M, int64_t h, int64_t f, int t, co
   TP_TRY(check_shards(W1, t, f / t, "W1"));
   TP_TRY(check_shards(W2, t, h, "W2"));
   TP_TRY(check_bias_array(b1, t, "b1"));
+  if (dtype == TP_BF16 && is_f16(W1)) return fail(TP_ERR_INVALID_ARG, "W1 must have X's dtype (bf16)");
+  if (dtype == TP_FP32 && (W1[0].dtype != TP_BF16 || W2[0].dtype != TP_BF16))
+    return fail(TP_ERR_INVALID_ARG, "fp32 FFN: leave the shards' dtype field at 0");
   const size_t need = tp_ffn_workspace_bytes(M, h, f, t, dtype, mode);
   if (need && (!ws || ws_bytes < need))
     return fail(TP_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws ? ws_bytes : 0);
@@ -349,9 +364,11 @@ tp_status attn_bf16(const void* X, int B, int S, int h, int H, int d, int t, con
   {
     GemmArgs a;
     memset(&a, 0, sizeof(a));
-    TP_TRY(make_tmap_bf16_2d(&a.tmA, X, h, M, static_cast<uint64_t>(h) * 2, 64, GEMM_BM));
+    const int f16 = is_f16(Wqkv);  // X has Wqkv's dtype
+    TP_TRY(make_tmap_2d(&a.tmA, X, f16, h, M, static_cast<uint64_t>(h) * 2, 64, GEMM_BM));
     for (int i = 0; i < t; ++i)
-      TP_TRY(make_tmap_bf16_2d(&a.tmB[i], Wqkv[i].ptr, ncol, h, Wqkv[i].ld * 2, 64, 64));
+      TP_TRY(make_tmap_2d(&a.tmB[i], Wqkv[i].ptr, f16, ncol, h, Wqkv[i].ld * 2, 64, 64));
+    a.ab_f16 = f16;
     a.M = static_cast<int>(M); a.N = static_cast<int>(ncol); a.Kg = h; a.G = t;
     a.concat = 0; a.a_k_per_group = 0;
     a.epi = EPI_QKV; a.act = ACT_NONE;
@@ -367,7 +384,8 @@ tp_status attn_bf16(const void* X, int B, int S, int h, int H, int d, int t, con
     TP_TRY(make_tmap_attn(&a.tmQ, w.q, B * H, S, d));
     TP_TRY(make_tmap_attn(&a.tmK, w.k, B * H, S, d));
     TP_TRY(make_tmap_attn(&a.tmV, w.v, B * H, S, d));
-    a.O = w.o; a.B = B; a.S = S; a.H = H; a.d = d; a.causal = causal; a.head0 = 0;
+    a.O = w.o; a.o_f16 = is_f16(Wo);
+    a.B = B; a.S = S; a.H = H; a.d = d; a.causal = causal; a.head0 = 0;
     a.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(d));
     a.status = device_status_ptr(); a.wait_limit_ns = wait_limit_ns();
     TP_TRY(launch_attention(a, stream));
@@ -390,6 +408,7 @@ tp_status validate_attn(const void* X, int B, int S, int h, int H, int d, int t,
   TP_TRY(check_shards(Wqkv, t, 3LL * (H / t) * d, "Wqkv"));
   TP_TRY(check_shards(Wo, t, h, "Wo"));
   TP_TRY(check_bias_array(bqkv, t, "bqkv"));
+  if (is_f16(Wqkv)) return fail(TP_ERR_INVALID_ARG, "Wqkv must have X's dtype (bf16)");
   const size_t need = attn_ws_bytes_i(B, S, h, H, d, t, mode);
   if (!ws || ws_bytes < need) return fail(TP_ERR_WORKSPACE, "workspace of %zu bytes needed", need);
   if (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN) return fail(TP_ERR_INVALID_ARG, "workspace not 256-byte aligned");
@@ -444,7 +463,8 @@ tp_status tp_column_linear_forward(const void* X, int64_t M, int64_t k, int64_t 
   TP_TRY(check_bias_array(b, t, "b"));
   if (M == 0) return TP_OK;
   const int kact = act == -1 ? ACT_NONE : (act == TP_ACT_GELU ? ACT_GELU : ACT_RELU);
-  return run_column(X, M, k, n / t, t, W, b, kact, out, n, static_cast<cudaStream_t>(stream));
+  return run_column(X, M, k, n / t, t, W, b, kact, out, is_f16(W) ? OUT_F16 : OUT_BF16, n,
+                    static_cast<cudaStream_t>(stream));
 }
 
 size_t tp_row_linear_workspace_bytes(int64_t M, int64_t n, int t, tp_reduce_mode mode) {
@@ -539,17 +559,18 @@ tp_status tp_layer_forward(const void* X, int B, int S, int h, int heads, int d,
   float* h1 = reinterpret_cast<float*>(p + a1b);
   uint16_t* a2 = reinterpret_cast<uint16_t*>(p + a1b + h1b);
   void* rest = p + a1b + h1b + a1b;
-  // h1 = X + Attn(LN1(X)), kept in fp32
-  TP_TRY(launch_layernorm(X, 0, ln1_g, ln1_b, M, h, eps, a1, s));
+  // h1 = X + Attn(LN1(X)), kept in fp32; LN1's output takes Wqkv's dtype
+  TP_TRY(launch_layernorm(X, 0, ln1_g, ln1_b, M, h, eps, a1, is_f16(Wqkv), s));
   TP_TRY(attn_bf16(a1, B, S, h, heads, d, t, Wqkv, bqkv, Wo, bo, X, 0, causal ? 1 : 0, h1, 1, mode, rest, s));
-  // out = h1 + FFN(LN2(h1))
-  TP_TRY(launch_layernorm(h1, 1, ln2_g, ln2_b, M, h, eps, a2, s));
+  // out = h1 + FFN(LN2(h1)); LN2's output takes W1's dtype
+  TP_TRY(launch_layernorm(h1, 1, ln2_g, ln2_b, M, h, eps, a2, is_f16(W1), s));
   return ffn_bf16(a2, M, h, f, t, W1, b1, W2, b2, h1, 1, out, 0, mode, ACT_GELU, rest, s);
 }
 
 tp_status tp_layernorm_forward(const void* x, tp_dtype in_dtype, const void* gamma, const void* beta, int64_t M,
-                               int64_t h, float eps, void* y, tp_stream_t stream) {
-  if (in_dtype != TP_BF16 && in_dtype != TP_FP32) return fail(TP_ERR_INVALID_ARG, "unknown dtype");
+                               int64_t h, float eps, void* y, tp_dtype out_dtype, tp_stream_t stream) {
+  if (in_dtype != TP_BF16 && in_dtype != TP_FP32) return fail(TP_ERR_INVALID_ARG, "unknown input dtype");
+  if (out_dtype != TP_BF16 && out_dtype != TP_FP16) return fail(TP_ERR_INVALID_ARG, "unknown output dtype");
   if (M < 0 || h <= 0) return fail(TP_ERR_INVALID_ARG, "bad sizes");
   if (h % 8) return fail(TP_ERR_UNSUPPORTED, "h %% 8 != 0");
   if (h > 49152) return fail(TP_ERR_UNSUPPORTED, "h > 49152");
@@ -559,7 +580,8 @@ tp_status tp_layernorm_forward(const void* x, tp_dtype in_dtype, const void* gam
   TP_TRY(check_ptr(gamma, "gamma", false));
   TP_TRY(check_ptr(beta, "beta", false));
   if (M > 0x7FFFFFFF) return fail(TP_ERR_UNSUPPORTED, "too many rows");
-  return launch_layernorm(x, in_dtype == TP_FP32, gamma, beta, M, h, eps, y, static_cast<cudaStream_t>(stream));
+  return launch_layernorm(x, in_dtype == TP_FP32, gamma, beta, M, h, eps, y, out_dtype == TP_FP16,
+                          static_cast<cudaStream_t>(stream));
 }
 
 tp_status tp_reduce_partials(const float* P, int t, int64_t M, int64_t h, const void* bias, const void* residual,

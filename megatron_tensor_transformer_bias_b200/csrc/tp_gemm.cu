@@ -35,7 +35,8 @@ constexpr int TMEM_COLS = NUM_ACC * BN;             // 512
 constexpr int THREADS = 192;
 constexpr int EPI_THREADS = 128;
 constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
-constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, /*a_mn=*/0, /*b_mn=*/1);
+constexpr uint32_t IDESC_BF16 = idesc_bf16_f32(BM, BN, /*a_mn=*/0, /*b_mn=*/1);
+constexpr uint32_t IDESC_F16 = idesc_f16_f32(BM, BN, /*a_mn=*/0, /*b_mn=*/1);
 
 struct TileCoord {
   int g, m_blk, n_blk;
@@ -92,17 +93,39 @@ __device__ __forceinline__ void store_bf16x32(void* p, const float (&v)[32]) {
   }
 }
 
+__device__ __forceinline__ void store_f16x32(void* p, const float (&v)[32]) {
+  uint4* q = reinterpret_cast<uint4*>(p);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint4 u;
+    u.x = pack_f16x2(v[i * 8 + 0], v[i * 8 + 1]);
+    u.y = pack_f16x2(v[i * 8 + 2], v[i * 8 + 3]);
+    u.z = pack_f16x2(v[i * 8 + 4], v[i * 8 + 5]);
+    u.w = pack_f16x2(v[i * 8 + 6], v[i * 8 + 7]);
+    q[i] = u;
+  }
+}
+
 __device__ __forceinline__ void store_f32x32(void* p, const float (&v)[32]) {
   float4* q = reinterpret_cast<float4*>(p);
 #pragma unroll
   for (int i = 0; i < 8; ++i) q[i] = make_float4(v[i * 4], v[i * 4 + 1], v[i * 4 + 2], v[i * 4 + 3]);
 }
 
+__device__ __forceinline__ void store_x32(void* base, int64_t idx, int out_type, const float (&v)[32]) {
+  if (out_type == OUT_F32)
+    store_f32x32(static_cast<float*>(base) + idx, v);
+  else if (out_type == OUT_F16)
+    store_f16x32(static_cast<uint16_t*>(base) + idx, v);
+  else
+    store_bf16x32(static_cast<uint16_t*>(base) + idx, v);
+}
+
 // One 32-column chunk of one accumulator row: apply the epilogue and store.
 __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, const TileCoord& tc, int row, int n,
                                                float (&v)[32]) {
   switch (a.epi) {
-    case EPI_ACT_BF16: {
+    case EPI_ACT: {
       if (a.bias_g[tc.g]) {
         float b[32];
         load_bf16x32(static_cast<const uint16_t*>(a.bias_g[tc.g]) + n, b);
@@ -111,9 +134,8 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, const TileCoor
       }
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] = act_apply(v[j], a.act);
-      uint16_t* o = static_cast<uint16_t*>(a.out) + static_cast<int64_t>(row) * a.ld_out +
-                    static_cast<int64_t>(tc.g) * a.out_col_per_group + n;
-      store_bf16x32(o, v);
+      store_x32(a.out, static_cast<int64_t>(row) * a.ld_out + static_cast<int64_t>(tc.g) * a.out_col_per_group + n,
+                a.out_type, v);
       break;
     }
     case EPI_PARTIAL_F32: {
@@ -138,10 +160,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, const TileCoor
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] += r[j];
       }
-      if (a.out_fp32)
-        store_f32x32(static_cast<float*>(a.out) + static_cast<int64_t>(row) * a.ld_out + n, v);
-      else
-        store_bf16x32(static_cast<uint16_t*>(a.out) + static_cast<int64_t>(row) * a.ld_out + n, v);
+      store_x32(a.out, static_cast<int64_t>(row) * a.ld_out + n, a.out_type, v);
       break;
     }
     case EPI_QKV: {
@@ -161,7 +180,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, const TileCoor
       void* base = part == 0 ? a.q : (part == 1 ? a.k : a.v);
       uint16_t* o = static_cast<uint16_t*>(base) +
                     ((static_cast<int64_t>(b) * a.H + head) * a.S + s) * a.d + dd;
-      store_bf16x32(o, v);
+      store_f16x32(o, v);
       break;
     }
     default:
@@ -264,6 +283,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
+      const uint32_t idesc = a.ab_f16 ? IDESC_F16 : IDESC_BF16;
       const uint32_t sA_addr = smem_u32(sA);
       const uint32_t sB_addr = smem_u32(sB);
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
@@ -286,7 +306,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
             const uint64_t adesc = smem_desc_sw128(a_base + k * 32, 16, 1024);
             // B: N-major, advance 16 K-rows (2048 bytes); 64-column blocks 8 KB apart.
             const uint64_t bdesc = smem_desc_sw128(b_base + k * 16 * 128, B_BLOCK_BYTES, 1024);
-            mma_bf16_ss(d_tmem, adesc, bdesc, IDESC, (it > 0 || k > 0) ? 1u : 0u);
+            mma_bf16_ss(d_tmem, adesc, bdesc, idesc, (it > 0 || k > 0) ? 1u : 0u);
           }
           mma_commit(&empty_bar[stage]);  // frees the smem stage once these MMAs finish
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }

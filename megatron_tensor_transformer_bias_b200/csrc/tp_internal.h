@@ -23,11 +23,14 @@ constexpr int GEMM_BN = 256;
 constexpr int GEMM_BK = 64;
 
 enum GemmEpilogue : int {
-  EPI_ACT_BF16 = 0,    // out[:, g*ncol + n] = act(acc + bias_g[n]) as bf16   (column-parallel layer)
+  EPI_ACT = 0,         // out[:, g*ncol + n] = act(acc + bias_g[n])            (column-parallel layer)
   EPI_PARTIAL_F32 = 1, // P[g][m, n] = acc as fp32                              (row layer, partials)
   EPI_BIAS_RESID = 2,  // out[m, n] = acc + bias[n] + resid[m, n]              (row layer, fused reduce)
-  EPI_QKV = 3,         // scatter acc (+ bias_g) to Q/K/V [B, H, S, d] bf16     (QKV column layer)
+  EPI_QKV = 3,         // scatter acc (+ bias_g) to Q/K/V [B, H, S, d] fp16     (QKV column layer)
 };
+
+// Element type of an epilogue output.
+enum OutType : int { OUT_BF16 = 0, OUT_F32 = 1, OUT_F16 = 2 };
 
 enum Activation : int { ACT_NONE = 0, ACT_GELU = 1, ACT_RELU = 2 };
 
@@ -38,11 +41,12 @@ struct __align__(64) GemmArgs {
   int concat;                           // 1: one tile sums all G K-slices in order g = 0..G-1
   int a_k_per_group;                    // column offset of group g's K-slice in A (elements)
   int epi, act;
+  int ab_f16;                           // A and B operands are fp16 (else bf16)
   void* out;
   int64_t ld_out;                       // elements
   int64_t out_col_per_group;            // EPI_ACT_BF16: column offset of group g in out
   int64_t out_group_stride;             // EPI_PARTIAL_F32: elements between partials
-  int out_fp32;
+  int out_type;                         // OutType of EPI_ACT / EPI_BIAS_RESID
   const void* bias_g[TP_MAX_SHARDS];    // bf16 [N] per group, or null
   const void* bias;                     // bf16 [N] or null (EPI_BIAS_RESID)
   const void* resid;                    // [M, N] or null
@@ -56,10 +60,11 @@ struct __align__(64) GemmArgs {
 };
 
 struct AttnArgs {
-  CUtensorMap tmQ;   // Q [B*H*S, d] bf16, box {64, 128}, 128B swizzle
-  CUtensorMap tmK;   // K [B*H*S, d]
-  CUtensorMap tmV;   // V [B*H*S, d]
-  void* O;           // O [B*S, H*d] bf16 (head-major columns)
+  CUtensorMap tmQ;   // Q [B*H][S][d] fp16, box {64, 128, 1}, 128B swizzle
+  CUtensorMap tmK;   // K [B*H][S][d] fp16
+  CUtensorMap tmV;   // V [B*H][S][d] fp16
+  void* O;           // O [B*S, H*d] (head-major columns), bf16 or fp16
+  int o_f16;
   int B, S, H, d, causal;
   int head0;         // first head handled (head-group offset)
   float scale_log2;  // log2(e) / sqrt(d)
@@ -73,8 +78,9 @@ uint32_t* device_status_ptr();
 uint64_t wait_limit_ns();
 
 // Tensor-map construction (driver entry point fetched through the runtime).
-tp_status make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                            uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+// 2-byte element tensor maps (bf16 or fp16), 128-byte swizzle, zero fill out of bounds.
+tp_status make_tmap_2d(CUtensorMap* map, const void* base, int f16, uint64_t inner, uint64_t outer,
+                       uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
 
 // Kernel launchers.  All are asynchronous on `stream` and validate nothing:
 // the C-ABI layer has checked every argument before calling them.
@@ -84,7 +90,7 @@ tp_status launch_reduce_partials(const float* P, int t, int64_t M, int64_t h, co
                                  const void* resid, int resid_fp32, void* out, int out_fp32,
                                  cudaStream_t stream);
 tp_status launch_layernorm(const void* x, int in_fp32, const void* g, const void* b, int64_t M, int64_t h,
-                           float eps, void* y, cudaStream_t stream);
+                           float eps, void* y, int out_f16, cudaStream_t stream);
 tp_status launch_ffn_fp32(const float* X, int64_t M, int64_t h, int64_t f, int t, const tp_shard* W1,
                           const void* const* b1, const tp_shard* W2, const float* b2, const float* resid,
                           float* out, int act, float* Z, float* P, cudaStream_t stream);

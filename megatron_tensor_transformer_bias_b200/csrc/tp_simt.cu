@@ -73,7 +73,7 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return s;
 }
 
-template <bool IN_F32>
+template <bool IN_F32, bool OUT_F16>
 __global__ void __launch_bounds__(LN_THREADS) layernorm_kernel(const void* __restrict__ x,
                                                                const uint16_t* __restrict__ g,
                                                                const uint16_t* __restrict__ b, int64_t h,
@@ -122,10 +122,17 @@ __global__ void __launch_bounds__(LN_THREADS) layernorm_kernel(const void* __res
       o[j] = (row[c] - mean) * rstd * gg + bb;
     }
     uint4 u;
-    u.x = pack_bf16x2(o[0], o[1]);
-    u.y = pack_bf16x2(o[2], o[3]);
-    u.z = pack_bf16x2(o[4], o[5]);
-    u.w = pack_bf16x2(o[6], o[7]);
+    if (OUT_F16) {
+      u.x = pack_f16x2(o[0], o[1]);
+      u.y = pack_f16x2(o[2], o[3]);
+      u.z = pack_f16x2(o[4], o[5]);
+      u.w = pack_f16x2(o[6], o[7]);
+    } else {
+      u.x = pack_bf16x2(o[0], o[1]);
+      u.y = pack_bf16x2(o[2], o[3]);
+      u.z = pack_bf16x2(o[4], o[5]);
+      u.w = pack_bf16x2(o[6], o[7]);
+    }
     reinterpret_cast<uint4*>(y + r * h)[v] = u;
   }
 }
@@ -217,27 +224,26 @@ tp_status launch_reduce_partials(const float* P, int t, int64_t M, int64_t h, co
 }
 
 tp_status launch_layernorm(const void* x, int in_fp32, const void* g, const void* b, int64_t M, int64_t h,
-                           float eps, void* y, cudaStream_t stream) {
+                           float eps, void* y, int out_f16, cudaStream_t stream) {
   if (M == 0) return TP_OK;
   const size_t smem = static_cast<size_t>(h) * sizeof(float);
-  static int attr_set[64][2] = {{0}};
+  const int key = (in_fp32 ? 1 : 0) | (out_f16 ? 2 : 0);
+  void (*kern)(const void*, const uint16_t*, const uint16_t*, int64_t, float, uint16_t*) =
+      key == 0 ? layernorm_kernel<false, false>
+               : key == 1 ? layernorm_kernel<true, false> : key == 2 ? layernorm_kernel<false, true>
+                                                                     : layernorm_kernel<true, true>;
+  static int attr_set[64][4] = {{0}};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return TP_ERR_CUDA;
-  if (smem > 48 * 1024 && dev < 64 && !attr_set[dev][in_fp32]) {
-    cudaError_t e = in_fp32 ? cudaFuncSetAttribute(layernorm_kernel<true>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024)
-                            : cudaFuncSetAttribute(layernorm_kernel<false>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    if (e != cudaSuccess) return TP_ERR_CUDA;
-    attr_set[dev][in_fp32] = 1;
+  if (smem > 48 * 1024 && dev < 64 && !attr_set[dev][key]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) != cudaSuccess)
+      return TP_ERR_CUDA;
+    attr_set[dev][key] = 1;
   }
   trace_before(stream);
-  if (in_fp32)
-    layernorm_kernel<true><<<static_cast<unsigned>(M), LN_THREADS, smem, stream>>>(
-        x, static_cast<const uint16_t*>(g), static_cast<const uint16_t*>(b), h, eps, static_cast<uint16_t*>(y));
-  else
-    layernorm_kernel<false><<<static_cast<unsigned>(M), LN_THREADS, smem, stream>>>(
-        x, static_cast<const uint16_t*>(g), static_cast<const uint16_t*>(b), h, eps, static_cast<uint16_t*>(y));
+  kern<<<static_cast<unsigned>(M), LN_THREADS, smem, stream>>>(x, static_cast<const uint16_t*>(g),
+                                                               static_cast<const uint16_t*>(b), h, eps,
+                                                               static_cast<uint16_t*>(y));
   if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
   trace_after(stream, "layernorm");
   return TP_OK;

@@ -119,3 +119,10 @@ def sample_rows(M, n, seed=0, seq=None):
             chosen.append(r)
             seen.add(r)
     return sorted(chosen)
+
+
+def as_fp16(w):
+    """An fp16 copy of a bf16 weight (same values: bf16 -> fp16 is exact for every
+    |w| >= 2**-17 below 65504, which covers N(0, 0.02^2) weights but for about
+    3 in 10^4 entries, whose change is below 2**-25 in absolute value)."""
+    return w.to(torch.float16)

@@ -17,7 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libtpblock.so")
 
 TP_OK, TP_ERR_INVALID_ARG, TP_ERR_UNSUPPORTED, TP_ERR_WORKSPACE, TP_ERR_CUDA, TP_ERR_TIMEOUT = range(6)
-TP_BF16, TP_FP32 = 0, 1
+TP_BF16, TP_FP32, TP_FP16 = 0, 1, 2
 TP_REDUCE_FUSED, TP_REDUCE_PARTIALS = 0, 1
 TP_ACT_GELU, TP_ACT_RELU = 0, 1
 TP_MAX_SHARDS = 16
@@ -27,7 +27,8 @@ ACTS = {"gelu": TP_ACT_GELU, "relu": TP_ACT_RELU, None: -1, "none": -1}
 
 
 class Shard(ctypes.Structure):
-    _fields_ = [("ptr", ctypes.c_void_p), ("ld", ctypes.c_int64)]
+    _fields_ = [("ptr", ctypes.c_void_p), ("ld", ctypes.c_int64), ("dtype", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
 
 
 class TPError(RuntimeError):
@@ -56,7 +57,7 @@ _SIGS = {
     "tp_layer_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32, _i64, _i32, _i32]),
     "tp_layer_forward": (_i32, [_vp, _i32, _i32, _i32, _i32, _i32, _i64, _i32, _vp, _vp, _SP, _VPP, _SP, _vp, _vp,
                                 _vp, _SP, _VPP, _SP, _vp, _f32, _i32, _vp, _i32, _vp, _sz, _vp]),
-    "tp_layernorm_forward": (_i32, [_vp, _i32, _vp, _vp, _i64, _i64, _f32, _vp, _vp]),
+    "tp_layernorm_forward": (_i32, [_vp, _i32, _vp, _vp, _i64, _i64, _f32, _vp, _i32, _vp]),
     "tp_reduce_partials": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _i32, _vp, _vp]),
     "tp_get_device_status": (_i32, [_vp]),
     "tp_set_wait_limit_ns": (None, [_u64]),
@@ -119,6 +120,7 @@ def _shards(ws: Sequence[torch.Tensor]):
             raise ValueError("a shard must be a 2-D view with unit column stride")
         arr[i].ptr = w.data_ptr()
         arr[i].ld = w.stride(0)
+        arr[i].dtype = TP_FP16 if w.dtype == torch.float16 else TP_BF16
     return arr
 
 
@@ -144,6 +146,8 @@ def _dtype_code(t: torch.Tensor) -> int:
         return TP_BF16
     if t.dtype == torch.float32:
         return TP_FP32
+    if t.dtype == torch.float16:
+        return TP_FP16
     raise ValueError(f"unsupported dtype {t.dtype}")
 
 
@@ -259,7 +263,7 @@ def tp_layer_forward(X, B, S, heads, d, ln1_g, ln1_b, Wqkv, bqkv, Wo, bo, ln2_g,
 def tp_layernorm_forward(x, gamma, beta, eps, y, stream=None):
     M, h = x.shape
     _check(lib().tp_layernorm_forward(_ptr(_dev(x)), _dtype_code(x), _ptr(gamma), _ptr(beta), M, h, float(eps),
-                                      _ptr(_dev(y)), _stream(stream)))
+                                      _ptr(_dev(y)), _dtype_code(y), _stream(stream)))
     return y
 
 

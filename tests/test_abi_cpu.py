@@ -109,6 +109,21 @@ def test_ffn_shard_validation(L):
     assert _ffn(L, W2=bad) == tb.TP_ERR_INVALID_ARG and "W2[0]" in tb.last_error()
 
 
+def test_shard_dtype_validation(L):
+    bad = _sh(2, 1024)
+    bad[1].dtype = tb.TP_FP16
+    assert _ffn(L, W1=bad) == tb.TP_ERR_INVALID_ARG and "mix" in tb.last_error()
+    bad = _sh(2, 1024)
+    bad[0].dtype = bad[1].dtype = 7
+    assert _ffn(L, W1=bad) == tb.TP_ERR_INVALID_ARG and "dtype" in tb.last_error()
+    f16 = _sh(2, 1024)
+    f16[0].dtype = f16[1].dtype = tb.TP_FP16
+    assert _ffn(L, W1=f16) == tb.TP_ERR_INVALID_ARG and "W1 must have X's dtype" in tb.last_error()
+    w2 = _sh(2, 256)
+    w2[0].dtype = w2[1].dtype = tb.TP_FP16
+    assert _ffn(L, W2=w2) == tb.TP_ERR_WORKSPACE  # fp16 W2 is valid: fails only on the missing workspace
+
+
 def test_ffn_empty_is_ok_without_launch(L):
     # M = 0: valid, nothing to do, no device touched
     assert _ffn(L, M=0, ws=None) == tb.TP_OK
@@ -126,12 +141,16 @@ def test_attention_validation(L):
     assert call(X=None) == tb.TP_ERR_INVALID_ARG
     assert call() == tb.TP_ERR_WORKSPACE
     assert call(B=0) == tb.TP_OK
+    f16 = _sh(t, 3 * 2 * 128)
+    f16[0].dtype = f16[1].dtype = tb.TP_FP16
+    assert call(Wqkv=f16) == tb.TP_ERR_INVALID_ARG and "Wqkv must have X's dtype" in tb.last_error()
 
 
 def test_layer_and_building_block_validation(L):
-    assert L.tp_layernorm_forward(FAKE, 0, None, None, 4, 100, 1e-5, FAKE + 4096, None) == tb.TP_ERR_UNSUPPORTED
-    assert L.tp_layernorm_forward(FAKE, 0, None, None, 4, 128, 0.0, FAKE + 4096, None) == tb.TP_ERR_INVALID_ARG
-    assert L.tp_layernorm_forward(None, 0, None, None, 4, 128, 1e-5, FAKE, None) == tb.TP_ERR_INVALID_ARG
+    assert L.tp_layernorm_forward(FAKE, 0, None, None, 4, 100, 1e-5, FAKE + 4096, 0, None) == tb.TP_ERR_UNSUPPORTED
+    assert L.tp_layernorm_forward(FAKE, 0, None, None, 4, 128, 0.0, FAKE + 4096, 0, None) == tb.TP_ERR_INVALID_ARG
+    assert L.tp_layernorm_forward(None, 0, None, None, 4, 128, 1e-5, FAKE, 0, None) == tb.TP_ERR_INVALID_ARG
+    assert L.tp_layernorm_forward(FAKE, 0, None, None, 4, 128, 1e-5, FAKE, 1, None) == tb.TP_ERR_INVALID_ARG
     assert L.tp_reduce_partials(FAKE, 0, 4, 128, None, None, 0, FAKE, None) == tb.TP_ERR_INVALID_ARG
     assert L.tp_reduce_partials(FAKE, 2, 4, 126, None, None, 0, FAKE, None) == tb.TP_ERR_UNSUPPORTED
     assert L.tp_selftest_bounded_wait(0, None) == tb.TP_ERR_INVALID_ARG
