@@ -126,6 +126,23 @@ TP_API tp_status tp_ffn_forward_act(const void* X, int64_t M, int64_t h, int64_t
                              void* out, tp_dtype dtype, tp_reduce_mode mode, tp_activation act, void* ws,
                              size_t ws_bytes, tp_stream_t stream);
 
+/* FFN block for callers that cannot allocate device memory (no counterpart on
+ * the page: it exists for callers that run inside a host framework owning the
+ * whole device memory pool, or in loops where a cudaMalloc and its possible
+ * device synchronisation are not allowed).  Same math as tp_ffn_forward with
+ * GeLU, bf16 X/W1/W2 and the fused reduction, but act(Z) goes to a static
+ * 16 MiB device array inside the library instead of a workspace:
+ * M * f <= 8,388,608, else TP_ERR_UNSUPPORTED with the sizes in tp_last_error().
+ * The caller still passes every input and the output.  It calls no cudaMalloc
+ * or cudaFree.  Every call on a device shares that array, so calls that overlap
+ * on the GPU (e.g. on two streams) race; nothing in it needs to start at zero.
+ * The first call on each device looks up the array's device address: make it
+ * before any stream capture.  Each GPU that loads the library keeps the 16 MiB
+ * until the process exits. */
+TP_API tp_status tp_ffn_forward_noalloc(const void* X, int64_t M, int64_t h, int64_t f, int t, const tp_shard* W1,
+                                        const void* const* b1, const tp_shard* W2, const void* b2,
+                                        const void* residual, void* out, tp_stream_t stream);
+
 /* ------------------------------------------------------------------ parallel linears
  * Column-parallel linear alone ([TP-CR] step 1), bf16 or fp16 (W's dtype):
  *   out[:, i*n/t : (i+1)*n/t] = act(X W_i + b_i)   for i < t,

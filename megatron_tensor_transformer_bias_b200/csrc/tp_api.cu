@@ -85,6 +85,11 @@ uint32_t* device_status_ptr() {
 
 uint64_t wait_limit_ns() { return g_wait_limit_ns.load(); }
 
+tp_status set_error(tp_status s, const char* msg) {
+  t_last_error = msg;
+  return s;
+}
+
 void trace_before(cudaStream_t stream) {
   if (!t_trace_on || static_cast<int>(t_trace.size()) >= t_trace_cap) return;
   t_pending_start = pool_event(2 * t_trace.size());

@@ -96,6 +96,9 @@ tp_status launch_ffn_fp32(const float* X, int64_t M, int64_t h, int64_t f, int t
                           float* out, int act, float* Z, float* P, cudaStream_t stream);
 tp_status launch_selftest_wait(uint64_t limit_ns, cudaStream_t stream);
 
+// Record `msg` as the calling thread's tp_last_error() and return `s`.
+tp_status set_error(tp_status s, const char* msg);
+
 // Launch tracing (tp_trace_*): brackets each kernel launch with events.
 void trace_before(cudaStream_t stream);
 void trace_after(cudaStream_t stream, const char* name);

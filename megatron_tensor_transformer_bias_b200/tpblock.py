@@ -48,6 +48,7 @@ _SIGS = {
     "tp_ffn_forward": (_i32, [_vp, _i64, _i64, _i64, _i32, _SP, _VPP, _SP, _vp, _vp, _vp, _i32, _i32, _vp, _sz, _vp]),
     "tp_ffn_forward_act": (_i32, [_vp, _i64, _i64, _i64, _i32, _SP, _VPP, _SP, _vp, _vp, _vp, _i32, _i32, _i32, _vp,
                                   _sz, _vp]),
+    "tp_ffn_forward_noalloc": (_i32, [_vp, _i64, _i64, _i64, _i32, _SP, _VPP, _SP, _vp, _vp, _vp, _vp]),
     "tp_column_linear_forward": (_i32, [_vp, _i64, _i64, _i64, _i32, _SP, _VPP, _i32, _vp, _vp]),
     "tp_row_linear_workspace_bytes": (_sz, [_i64, _i64, _i32, _i32]),
     "tp_row_linear_forward": (_i32, [_vp, _i64, _i64, _i64, _i32, _SP, _vp, _vp, _vp, _i32, _vp, _sz, _vp]),
@@ -194,6 +195,18 @@ def tp_ffn_forward(X, W1, b1, W2, b2, residual, out, mode="fused", act="gelu", w
     s = lib().tp_ffn_forward_act(_ptr(X), M, h, f, t, _shards(W1), _ptr_array(b1), _shards(W2), _ptr(b2),
                                  _ptr(residual), _ptr(out), dt, m, ACTS[act], _ptr(ws), ws.numel(), _stream(stream))
     _check(s)
+    return out
+
+
+def tp_ffn_forward_noalloc(X, W1, b1, W2, b2, residual, out, stream=None):
+    """The FFN block (GeLU, bf16, fused reduction) with act(Z) in the library's static
+    16 MiB device scratch instead of a workspace, for callers that cannot allocate."""
+    _dev(X); _dev(out)
+    M, h = X.shape
+    t = len(W1)
+    f = sum(w.shape[1] for w in W1)
+    _check(lib().tp_ffn_forward_noalloc(_ptr(X), M, h, f, t, _shards(W1), _ptr_array(b1), _shards(W2), _ptr(b2),
+                                        _ptr(residual), _ptr(out), _stream(stream)))
     return out
 
 
