@@ -213,6 +213,13 @@ TP_API tp_status tp_layer_forward(const void* X, int B, int S, int h, int heads,
 TP_API tp_status tp_layernorm_forward(const void* x, tp_dtype in_dtype, const void* gamma, const void* beta, int64_t M,
                                int64_t h, float eps, void* y, tp_dtype out_dtype, tp_stream_t stream);
 
+/* The element-wise nonlinearity of step 1 alone ([TP-CR], the paragraph on
+ * where the nonlinearity fits), exactly as the column layer's epilogue applies
+ * it: y[i] = act(x[i]) for fp32 x, y of n elements (may alias).  GeLU is the
+ * exact z*Phi(z) with erfc from the published approximation of Numerical Recipes
+ * (fractional error < 1.2e-7); in fp32 within 4e-7 absolute of the exact value. */
+TP_API tp_status tp_activation_forward(const float* x, float* y, int64_t n, tp_activation act, tp_stream_t stream);
+
 /* Step 3 alone: out = sum_{i<t} P[i] + bias + residual in fixed order i = 0..t-1.
  * P [t, M, h] fp32 contiguous; bias [h] and residual [M, h] in `dtype` or NULL;
  * out [M, h] in `dtype`.  h % 4 == 0. */

@@ -602,6 +602,13 @@ tp_status tp_reduce_partials(const float* P, int t, int64_t M, int64_t h, const 
   return launch_reduce_partials(P, t, M, h, bias, f32, residual, f32, out, f32, static_cast<cudaStream_t>(stream));
 }
 
+tp_status tp_activation_forward(const float* x, float* y, int64_t n, tp_activation act, tp_stream_t stream) {
+  if (n < 0) return fail(TP_ERR_INVALID_ARG, "n must be >= 0");
+  if (act != TP_ACT_GELU && act != TP_ACT_RELU) return fail(TP_ERR_INVALID_ARG, "unknown activation %d", act);
+  if (n > 0 && (!x || !y)) return fail(TP_ERR_INVALID_ARG, "x or y is NULL");
+  return launch_act(x, y, n, act == TP_ACT_GELU ? ACT_GELU : ACT_RELU, static_cast<cudaStream_t>(stream));
+}
+
 tp_status tp_get_device_status(tp_stream_t stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return fail(TP_ERR_CUDA, "stream synchronisation failed: %s", cudaGetErrorString(cudaGetLastError()));

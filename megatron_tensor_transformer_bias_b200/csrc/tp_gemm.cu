@@ -17,6 +17,8 @@
 //   warps 2..5  epilogue: tcgen05.ld TMEM -> registers -> bias/act/residual -> global
 // A 4-stage shared-memory ring feeds the MMA; two 256-column TMEM accumulators let
 // the epilogue of one tile overlap the main loop of the next.
+#include <cstdlib>
+
 #include "tp_internal.h"
 #include "tp_ptx.cuh"
 
@@ -32,8 +34,8 @@ constexpr int B_STAGE_BYTES = BN * BK * 2;          // 32 KB
 constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
 constexpr int NUM_ACC = 2;
 constexpr int TMEM_COLS = NUM_ACC * BN;             // 512
-constexpr int THREADS = 192;
-constexpr int EPI_THREADS = 128;
+constexpr int EPI_WARPS = 8;                        // two per TMEM sub-partition, each owns half the columns
+constexpr int THREADS = 64 + 32 * EPI_WARPS;        // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
 constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
 constexpr uint32_t IDESC_BF16 = idesc_bf16_f32(BM, BN, /*a_mn=*/0, /*b_mn=*/1);
 constexpr uint32_t IDESC_F16 = idesc_f16_f32(BM, BN, /*a_mn=*/0, /*b_mn=*/1);
@@ -49,12 +51,6 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int tile, int
   c.n_blk = rest % n_tiles;
   c.g = a.concat ? 0 : rest / n_tiles;
   return c;
-}
-
-__device__ __forceinline__ float act_apply(float v, int act) {
-  if (act == ACT_GELU) return v * 0.5f * (1.0f + erff(v * 0.70710678118654752440f));
-  if (act == ACT_RELU) return fmaxf(v, 0.0f);
-  return v;
 }
 
 __device__ __forceinline__ void load_bf16x32(const void* p, float (&v)[32]) {
@@ -220,7 +216,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
     }
     for (int s = 0; s < NUM_ACC; ++s) {
       mbar_init(&acc_full[s], 1);
-      mbar_init(&acc_empty[s], EPI_THREADS);
+      mbar_init(&acc_empty[s], EPI_WARPS);  // one arrival per epilogue warp
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -241,6 +237,9 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
     if (lane == 0) {
       tma_prefetch_desc(&a.tmA);
       for (int g = 0; g < a.G; ++g) tma_prefetch_desc(&a.tmB[g]);
+      // both operands are re-read by several CTAs at about the same time: default L2 policy
+      const uint64_t pol_a = l2_policy_evict_normal();
+      const uint64_t pol_b = pol_a;
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
@@ -257,11 +256,12 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
           const int g = a.concat ? it / kb_per_group : tc.g;
           const int kb = a.concat ? it - g * kb_per_group : it;
           mbar_arrive_expect_tx(&full_bar[stage], STAGE_BYTES);
-          tma_load_2d(sA + stage * A_STAGE_BYTES, &a.tmA, &full_bar[stage], g * a.a_k_per_group + kb * BK, m0);
+          tma_load_2d_hint(sA + stage * A_STAGE_BYTES, &a.tmA, &full_bar[stage], g * a.a_k_per_group + kb * BK, m0,
+                           pol_a);
           uint8_t* b_dst = sB + stage * B_STAGE_BYTES;
 #pragma unroll
           for (int j = 0; j < BN / 64; ++j)
-            tma_load_2d(b_dst + j * B_BLOCK_BYTES, &a.tmB[g], &full_bar[stage], n0 + j * 64, kb * BK);
+            tma_load_2d_hint(b_dst + j * B_BLOCK_BYTES, &a.tmB[g], &full_bar[stage], n0 + j * 64, kb * BK, pol_b);
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -323,6 +323,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
     // ------------------------------------------------------------ epilogue (warps 2..5)
     const int sub = warp & 3;               // TMEM sub-partition this warp may access
     const int row_in_tile = sub * 32 + lane;
+    const int col_half = (warp - 2) / 4;    // columns [col_half*BN/2, +BN/2) of each tile
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -340,22 +341,32 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
       const int row = tc.m_blk * BM + row_in_tile;
       const int n0 = tc.n_blk * BN;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(acc * BN);
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        const int n = n0 + c * 32;
-        if (n >= a.N) break;  // uniform over the CTA: N is a multiple of 32
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(t_row + c * 32, r);
-        tmem_ld_wait();
-        if (row < a.M) {
-          float v[32];
+      // columns [c_begin*32, c_end*32) of the tile, clipped to N (a multiple of 32);
+      // the TMEM load of chunk c+1 is issued before chunk c is processed
+      const int c_begin = col_half * (BN / 64);
+      int c_end = (col_half + 1) * (BN / 64);
+      if (n0 + c_end * 32 > a.N) c_end = (a.N - n0) / 32;
+      if (c_begin < c_end) {
+        uint32_t r[2][32];
+        tmem_ld_32x32b_x32(t_row + c_begin * 32, r[0]);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          epilogue_chunk(a, tc, row, n, v);
+        for (int c = c_begin; c < c_begin + BN / 64; ++c) {
+          if (c >= c_end) break;
+          tmem_ld_wait();
+          const int cur = (c - c_begin) & 1;
+          if (c + 1 < c_end) tmem_ld_32x32b_x32(t_row + (c + 1) * 32, r[cur ^ 1]);
+          if (row < a.M) {
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[cur][j]);
+            epilogue_chunk(a, tc, row, n0 + c * 32, v);
+          }
         }
+        tmem_ld_wait();
       }
       tc_fence_before();
-      mbar_arrive(&acc_empty[acc]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
       if (++acc == NUM_ACC) { acc = 0; acc_phase ^= 1u; }
     }
   }
@@ -369,12 +380,291 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
   }
 }
 
+// ============================================================================ CTA-pair variant
+// Same roles and epilogues; a cluster of two CTAs computes a 256x256 tile with
+// tcgen05.mma.cta_group::2 (M=256, N=256, K=16) issued by the leader (rank 0).
+// Each CTA loads only its own operand halves -- A rows [rank*128, +128) and B
+// columns [rank*128, +128) of the tile -- so each SM streams 32 KB per 64-wide K
+// step instead of 48 KB.  Both CTAs' TMA loads count their bytes on the leader's
+// full barrier; the leader's commits arrive on both CTAs' empty / accumulator
+// barriers; both CTAs' epilogues arrive on the leader's accumulator-empty barrier.
+// No load is multicast.
+constexpr int P_ROWS = 2 * BM;                      // 256 rows per pair
+constexpr int P_STAGES = 6;
+constexpr int P_A_BYTES = BM * BK * 2;              // 16 KB per CTA
+constexpr int P_B_BYTES = (BN / 2) * BK * 2;        // 16 KB per CTA
+constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
+constexpr int P_SMEM_BYTES = 1024 + P_STAGES * P_STAGE_BYTES + 256;
+constexpr uint32_t P_IDESC_BF16 = idesc_bf16_f32(P_ROWS, BN, 0, 1);
+constexpr uint32_t P_IDESC_F16 = idesc_f16_f32(P_ROWS, BN, 0, 1);
+
+__global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_constant__ GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + P_STAGES * P_A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P_STAGES * P_STAGE_BYTES);
+  uint64_t* full_bar = bars;                             // [P_STAGES], used in the leader
+  uint64_t* empty_bar = bars + P_STAGES;                 // [P_STAGES], both CTAs
+  uint64_t* acc_full = bars + 2 * P_STAGES;              // [NUM_ACC], both CTAs
+  uint64_t* acc_empty = bars + 2 * P_STAGES + NUM_ACC;   // [NUM_ACC], used in the leader
+  uint64_t* drain_bar = bars + 2 * P_STAGES + 2 * NUM_ACC;
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cid = static_cast<int>(blockIdx.x >> 1);
+  const int nclusters = static_cast<int>(gridDim.x >> 1);
+
+  const int m_tiles = (a.M + P_ROWS - 1) / P_ROWS;
+  const int n_tiles = (a.N + BN - 1) / BN;
+  const int num_tiles = m_tiles * n_tiles * (a.concat ? 1 : a.G);
+  const int kb_per_group = a.Kg / BK;
+  const int k_iters = a.concat ? kb_per_group * a.G : kb_per_group;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int s = 0; s < NUM_ACC; ++s) {
+      mbar_init(&acc_full[s], 1);
+      mbar_init(&acc_empty[s], 2 * EPI_WARPS);  // one arrival per epilogue warp of each CTA
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_base_slot, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers of both CTAs initialised before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_base_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      tma_prefetch_desc(&a.tmA);
+      for (int g = 0; g < a.G; ++g) tma_prefetch_desc(&a.tmB[g]);
+      // both operands are re-read by several CTAs at about the same time: default L2 policy
+      const uint64_t pol_a = l2_policy_evict_normal();
+      const uint64_t pol_b = pol_a;
+      const uint32_t full0_leader = mapa_shared(smem_u32(&full_bar[0]), 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int tile = cid; tile < num_tiles && ok; tile += nclusters) {
+        const TileCoord tc = tile_coord(a, tile, m_tiles, n_tiles);
+        const int m0 = tc.m_blk * P_ROWS + static_cast<int>(rank) * BM;
+        const int n0 = tc.n_blk * BN + static_cast<int>(rank) * (BN / 2);
+        for (int it = 0; it < k_iters; ++it) {
+          if (*abort_flag) { ok = false; break; }
+          if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, a.wait_limit_ns, a.status, WAIT_SITE_PRODUCER)) {
+            *abort_flag = 1; ok = false; break;
+          }
+          const int g = a.concat ? it / kb_per_group : tc.g;
+          const int kb = a.concat ? it - g * kb_per_group : it;
+          const uint32_t fb = full0_leader + static_cast<uint32_t>(stage) * 8u;
+          if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * P_STAGE_BYTES);
+          tma_load_2d_pair(sA + stage * P_A_BYTES, &a.tmA, fb, g * a.a_k_per_group + kb * BK, m0, pol_a);
+          uint8_t* b_dst = sB + stage * P_B_BYTES;
+          tma_load_2d_pair(b_dst, &a.tmB[g], fb, n0, kb * BK, pol_b);
+          tma_load_2d_pair(b_dst + B_BLOCK_BYTES, &a.tmB[g], fb, n0 + 64, kb * BK, pol_b);
+          ++issued;
+          if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // Our copies are in flight until the leader's MMAs have consumed their stage:
+      // wait for the consumption of the last min(issued, P_STAGES) stages.
+      const int pending = issued < P_STAGES ? issued : P_STAGES;
+      int s = stage;
+      uint32_t ph = phase;
+      for (int i = 0; i < pending; ++i) {
+        if (--s < 0) { s = P_STAGES - 1; ph ^= 1u; }
+        mbar_wait_bounded(&empty_bar[s], ph, a.wait_limit_ns, a.status, WAIT_SITE_PRODUCER);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (lane == 0 && leader) {
+      const uint32_t idesc = a.ab_f16 ? P_IDESC_F16 : P_IDESC_BF16;
+      const uint32_t sA_addr = smem_u32(sA);
+      const uint32_t sB_addr = smem_u32(sB);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = cid; tile < num_tiles && ok; tile += nclusters) {
+        if (!mbar_wait_bounded(&acc_empty[acc], acc_phase ^ 1u, a.wait_limit_ns, a.status, WAIT_SITE_MMA_ACC)) {
+          *abort_flag = 1; ok = false; break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int it = 0; it < k_iters; ++it) {
+          if (*abort_flag) { ok = false; break; }
+          if (!mbar_wait_bounded(&full_bar[stage], phase, a.wait_limit_ns, a.status, WAIT_SITE_MMA_FULL)) {
+            *abort_flag = 1; ok = false; break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = sA_addr + stage * P_A_BYTES;
+          const uint32_t b_base = sB_addr + stage * P_B_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t adesc = smem_desc_sw128(a_base + k * 32, 16, 1024);
+            const uint64_t bdesc = smem_desc_sw128(b_base + k * 16 * 128, B_BLOCK_BYTES, 1024);
+            mma_pair_ss(d_tmem, adesc, bdesc, idesc, (it > 0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit_pair_mask(&empty_bar[stage], 0x3);  // frees this stage in both CTAs
+          if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit_pair_mask(&acc_full[acc], 0x3);       // accumulator ready in both CTAs
+        if (++acc == NUM_ACC) { acc = 0; acc_phase ^= 1u; }
+      }
+      mma_commit_pair_local(drain_bar);
+      mbar_wait_bounded(drain_bar, 0, a.wait_limit_ns, a.status, WAIT_SITE_MMA_ACC);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5 of both CTAs)
+    const int sub = warp & 3;
+    const int row_in_tile = static_cast<int>(rank) * BM + sub * 32 + lane;
+    const int col_half = (warp - 2) / 4;    // columns [col_half*BN/2, +BN/2) of each tile
+    const uint32_t acc_empty0_leader = mapa_shared(smem_u32(&acc_empty[0]), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = cid; tile < num_tiles; tile += nclusters) {
+      if (*abort_flag) break;
+      const bool ready = __all_sync(0xffffffffu,
+                                    mbar_wait_bounded(&acc_full[acc], acc_phase, a.wait_limit_ns, a.status,
+                                                      WAIT_SITE_EPILOGUE));
+      if (!ready) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const TileCoord tc = tile_coord(a, tile, m_tiles, n_tiles);
+      const int row = tc.m_blk * P_ROWS + row_in_tile;
+      const int n0 = tc.n_blk * BN;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      // columns [c_begin*32, c_end*32) of the tile, clipped to N (a multiple of 32);
+      // the TMEM load of chunk c+1 is issued before chunk c is processed
+      const int c_begin = col_half * (BN / 64);
+      int c_end = (col_half + 1) * (BN / 64);
+      if (n0 + c_end * 32 > a.N) c_end = (a.N - n0) / 32;
+      if (c_begin < c_end) {
+        uint32_t r[2][32];
+        tmem_ld_32x32b_x32(t_row + c_begin * 32, r[0]);
+#pragma unroll
+        for (int c = c_begin; c < c_begin + BN / 64; ++c) {
+          if (c >= c_end) break;
+          tmem_ld_wait();
+          const int cur = (c - c_begin) & 1;
+          if (c + 1 < c_end) tmem_ld_32x32b_x32(t_row + (c + 1) * 32, r[cur ^ 1]);
+          if (row < a.M) {
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[cur][j]);
+            epilogue_chunk(a, tc, row, n0 + c * 32, v);
+          }
+        }
+        tmem_ld_wait();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty0_leader + static_cast<uint32_t>(acc) * 8u);
+      if (++acc == NUM_ACC) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();  // the leader's MMAs and the remote arrives are done in both CTAs
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
 }  // namespace
+
+// CTA pairs are the default; TPB_GEMM_PAIRS=0 selects the one-CTA kernel.
+static bool gemm_use_pairs() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("TPB_GEMM_PAIRS");
+    v = (e && e[0] == '0') ? 0 : 1;
+  }
+  return v == 1;
+}
+
+static int g_pair_clusters[64] = {0};
+
+// Largest number of co-resident CTA pairs for the pair kernel on this device.
+static int pair_clusters(int dev) {
+  if (dev < 0 || dev >= 64) return 0;
+  if (g_pair_clusters[dev]) return g_pair_clusters[dev];
+  if (cudaFuncSetAttribute(tp_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES) !=
+      cudaSuccess)
+    return -1;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * (sm_count() / 2), 1, 1);
+  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.dynamicSmemBytes = P_SMEM_BYTES;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, tp_gemm_pair_kernel, &cfg) != cudaSuccess || n <= 0) return -1;
+  g_pair_clusters[dev] = n;
+  return n;
+}
+
+static tp_status launch_gemm_pair(const GemmArgs& a, cudaStream_t stream, const char* name, int dev) {
+  const int nclusters_max = pair_clusters(dev);
+  if (nclusters_max <= 0) return TP_ERR_CUDA;
+  const int m_tiles = (a.M + P_ROWS - 1) / P_ROWS;
+  const int n_tiles = (a.N + BN - 1) / BN;
+  const long long tiles = 1LL * m_tiles * n_tiles * (a.concat ? 1 : a.G);
+  if (tiles <= 0) return TP_OK;
+  const int nclusters = static_cast<int>(tiles < nclusters_max ? tiles : nclusters_max);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * nclusters, 1, 1);
+  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.dynamicSmemBytes = P_SMEM_BYTES;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  trace_before(stream);
+  if (cudaLaunchKernelEx(&cfg, tp_gemm_pair_kernel, a) != cudaSuccess) return TP_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
+  trace_after(stream, name);
+  return TP_OK;
+}
 
 tp_status launch_gemm(const GemmArgs& a, cudaStream_t stream, const char* name) {
   static int attr_set[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return TP_ERR_CUDA;
+  if (gemm_use_pairs()) return launch_gemm_pair(a, stream, name, dev);
   if (dev < 64 && !attr_set[dev]) {
     if (cudaFuncSetAttribute(tp_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
         cudaSuccess)

@@ -95,6 +95,7 @@ tp_status launch_ffn_fp32(const float* X, int64_t M, int64_t h, int64_t f, int t
                           const void* const* b1, const tp_shard* W2, const float* b2, const float* resid,
                           float* out, int act, float* Z, float* P, cudaStream_t stream);
 tp_status launch_selftest_wait(uint64_t limit_ns, cudaStream_t stream);
+tp_status launch_act(const float* x, float* y, int64_t n, int act, cudaStream_t stream);
 
 // Record `msg` as the calling thread's tp_last_error() and return `s`.
 tp_status set_error(tp_status s, const char* msg);

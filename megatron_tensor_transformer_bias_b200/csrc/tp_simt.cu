@@ -172,10 +172,17 @@ __global__ void __launch_bounds__(SG * SG) f32_gemm_kernel(const float* __restri
   }
   if (row < M && col < N) {
     if (sp.bias[z]) acc += sp.bias[z][col];
-    if (act == ACT_GELU) acc = acc * 0.5f * (1.0f + erff(acc * 0.70710678118654752440f));
-    else if (act == ACT_RELU) acc = fmaxf(acc, 0.f);
+    acc = act_apply(acc, act);
     C[z * c_mat_step + z * c_col_step + static_cast<int64_t>(row) * ldc + col] = acc;
   }
+}
+
+// ---------------------------------------------------------------- element-wise nonlinearity
+__global__ void __launch_bounds__(256) act_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n,
+                                                  int act) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    y[i] = act_apply(x[i], act);
 }
 
 // ---------------------------------------------------------------- self-test
@@ -279,6 +286,18 @@ tp_status launch_ffn_fp32(const float* X, int64_t M, int64_t h, int64_t f, int t
   trace_after(stream, "f32_row_gemm");
   // Step 3: out = sum_i P[i] + b2 + residual
   return launch_reduce_partials(P, t, M, h, b2, 1, resid, 1, out, 1, stream);
+}
+
+tp_status launch_act(const float* x, float* y, int64_t n, int act, cudaStream_t stream) {
+  if (n == 0) return TP_OK;
+  int64_t blocks = (n + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+  if (blocks > cap) blocks = cap;
+  trace_before(stream);
+  act_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(x, y, n, act);
+  if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
+  trace_after(stream, "activation");
+  return TP_OK;
 }
 
 tp_status launch_selftest_wait(uint64_t limit_ns, cudaStream_t stream) {

@@ -60,6 +60,7 @@ _SIGS = {
                                 _vp, _SP, _VPP, _SP, _vp, _f32, _i32, _vp, _i32, _vp, _sz, _vp]),
     "tp_layernorm_forward": (_i32, [_vp, _i32, _vp, _vp, _i64, _i64, _f32, _vp, _i32, _vp]),
     "tp_reduce_partials": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _i32, _vp, _vp]),
+    "tp_activation_forward": (_i32, [_vp, _vp, _i64, _i32, _vp]),
     "tp_get_device_status": (_i32, [_vp]),
     "tp_set_wait_limit_ns": (None, [_u64]),
     "tp_selftest_bounded_wait": (_i32, [_u64, _vp]),
@@ -277,6 +278,14 @@ def tp_layernorm_forward(x, gamma, beta, eps, y, stream=None):
     M, h = x.shape
     _check(lib().tp_layernorm_forward(_ptr(_dev(x)), _dtype_code(x), _ptr(gamma), _ptr(beta), M, h, float(eps),
                                       _ptr(_dev(y)), _dtype_code(y), _stream(stream)))
+    return y
+
+
+def tp_activation_forward(x, y, act="gelu", stream=None):
+    """y = act(x) element-wise (fp32), as the column layer's epilogue applies it."""
+    if x.dtype != torch.float32 or y.dtype != torch.float32:
+        raise ValueError("fp32 tensors expected")
+    _check(lib().tp_activation_forward(_ptr(_dev(x)), _ptr(_dev(y)), x.numel(), ACTS[act], _stream(stream)))
     return y
 
 

@@ -154,6 +154,10 @@ def test_layer_and_building_block_validation(L):
     assert L.tp_reduce_partials(FAKE, 0, 4, 128, None, None, 0, FAKE, None) == tb.TP_ERR_INVALID_ARG
     assert L.tp_reduce_partials(FAKE, 2, 4, 126, None, None, 0, FAKE, None) == tb.TP_ERR_UNSUPPORTED
     assert L.tp_selftest_bounded_wait(0, None) == tb.TP_ERR_INVALID_ARG
+    assert L.tp_activation_forward(None, FAKE, 10, 0, None) == tb.TP_ERR_INVALID_ARG
+    assert L.tp_activation_forward(FAKE, FAKE, 10, 7, None) == tb.TP_ERR_INVALID_ARG
+    assert L.tp_activation_forward(FAKE, FAKE, -1, 0, None) == tb.TP_ERR_INVALID_ARG
+    assert L.tp_activation_forward(None, None, 0, 0, None) == tb.TP_OK
     assert L.tp_trace_enable(0) == tb.TP_ERR_INVALID_ARG
     assert L.tp_column_linear_forward(FAKE, 4, 100, 128, 1, _sh(1, 128), None, -1, FAKE, None) == tb.TP_ERR_UNSUPPORTED
     assert L.tp_row_linear_forward(FAKE, 4, 128, 128, 1, _sh(1, 128), None, None, FAKE + 4096, 1, None, 0,

@@ -80,3 +80,26 @@ def test_launch_trace_names_kernels():
     names = [n for n, _ in recs]
     assert names == ["gemm_column_act", "gemm_row_partials", "reduce_partials"]
     assert all(ms > 0 for _, ms in recs)
+
+
+def test_activation_matches_exact_gelu_and_relu():
+    """The column layer's nonlinearity in fp32 against the fp64 oracle: the published erfc
+    approximation it uses has fractional error < 1.2e-7; in fp32 the GeLU stays within
+    4e-7 absolute (2e-5 relative in the far negative tail)."""
+    g = torch.Generator(device=DEV).manual_seed(41)
+    x = torch.cat([torch.linspace(-14, 14, 200001, device=DEV),
+                   torch.randn(100000, generator=g, device=DEV) * 3,
+                   torch.tensor([0.0, -0.0, 1.0, -1.0, 2.0, 0.5, 1e-30, -1e-30, 40.0, -40.0], device=DEV)])
+    y = torch.empty_like(x)
+    tb.tp_activation_forward(x, y, "gelu")
+    ref = oracle.gelu(to64(x))
+    err = np.abs(to64(y) - ref)
+    assert (err <= 1e-6 + 3e-5 * np.abs(ref)).all(), float(err.max())
+    # table values of the exact GeLU, x * Phi(x)
+    yy = to64(y)[-10:]
+    assert yy[0] == 0.0 and yy[1] == 0.0
+    assert abs(yy[2] - 0.8413447460685429) < 2e-7 and abs(yy[3] + (1 - 0.8413447460685429)) < 2e-7
+    assert abs(yy[4] - 2 * 0.9772498680518208) < 4e-7 and abs(yy[5] - 0.5 * 0.6914624612740131) < 2e-7
+    assert yy[8] == 40.0 and yy[9] == 0.0
+    tb.tp_activation_forward(x, y, "relu")
+    assert torch.equal(y, torch.clamp(x, min=0.0))
