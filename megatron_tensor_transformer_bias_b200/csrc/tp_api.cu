@@ -139,6 +139,21 @@ tp_status make_tmap_2d(CUtensorMap* map, const void* base, int f16, uint64_t inn
   return TP_OK;
 }
 
+tp_status make_tmap_out(CUtensorMap* map, void* base, int f16, uint64_t cols, uint64_t rows,
+                        uint64_t row_stride_bytes) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled(out) failed (%d)", static_cast<int>(r));
+  return TP_OK;
+}
+
 static tp_status make_tmap_f16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                                    uint64_t s1_bytes, uint64_t s2_bytes, uint32_t b0, uint32_t b1) {
   EncodeTiledFn enc = encode_fn();
@@ -241,6 +256,10 @@ tp_status run_column(const void* X, int64_t M, int64_t k, int64_t ncol, int t, c
   a.concat = 0; a.a_k_per_group = 0;
   a.epi = EPI_ACT; a.act = act; a.ab_f16 = f16;
   a.out = out; a.ld_out = ld_out; a.out_col_per_group = ncol; a.out_type = out_type;
+  if (out_type != OUT_F32) {
+    TP_TRY(make_tmap_out(&a.tmOut, out, out_type == OUT_F16, static_cast<uint64_t>(ld_out), M, ld_out * 2));
+    a.tma_store = 1;
+  }
   for (int i = 0; i < t; ++i) a.bias_g[i] = b ? b[i] : nullptr;
   a.status = device_status_ptr(); a.wait_limit_ns = wait_limit_ns();
   return launch_gemm(a, stream, "gemm_column_act");
@@ -264,6 +283,10 @@ tp_status run_row(const void* A, int64_t M, int64_t kg, int64_t n, int t, const 
     a.concat = 1;
     a.epi = EPI_BIAS_RESID;
     a.out = out; a.ld_out = n; a.out_type = out_fp32 ? OUT_F32 : OUT_BF16;
+    if (!out_fp32) {
+      TP_TRY(make_tmap_out(&a.tmOut, out, 0, static_cast<uint64_t>(n), M, n * 2));
+      a.tma_store = 1;
+    }
     a.bias = bias; a.resid = resid; a.ld_resid = n; a.resid_fp32 = resid_fp32;
     return launch_gemm(a, stream, "gemm_row_fused_reduce");
   }

@@ -36,7 +36,8 @@ constexpr int NUM_ACC = 2;
 constexpr int TMEM_COLS = NUM_ACC * BN;             // 512
 constexpr int EPI_WARPS = 8;                        // two per TMEM sub-partition, each owns half the columns
 constexpr int THREADS = 64 + 32 * EPI_WARPS;        // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+constexpr int STAGING_BYTES = EPI_WARPS * 2 * 2048;   // two 32x32 16-bit buffers per epilogue warp
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + 256;
 constexpr uint32_t IDESC_BF16 = idesc_bf16_f32(BM, BN, /*a_mn=*/0, /*b_mn=*/1);
 constexpr uint32_t IDESC_F16 = idesc_f16_f32(BM, BN, /*a_mn=*/0, /*b_mn=*/1);
 
@@ -117,6 +118,65 @@ __device__ __forceinline__ void store_x32(void* base, int64_t idx, int out_type,
     store_bf16x32(static_cast<uint16_t*>(base) + idx, v);
 }
 
+// Bias / nonlinearity / residual of one 32-column chunk for the epilogues whose
+// 16-bit output leaves through a TMA store (EPI_ACT, EPI_BIAS_RESID).  Rows at or
+// beyond M still run (their values are clipped by the store) but read no residual.
+__device__ __forceinline__ void epilogue_math(const GemmArgs& a, const TileCoord& tc, int row, int n, float (&v)[32]) {
+  const void* bias = a.epi == EPI_ACT ? a.bias_g[tc.g] : a.bias;
+  if (bias) {
+    float b[32];
+    load_bf16x32(static_cast<const uint16_t*>(bias) + n, b);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] += b[j];
+  }
+  if (a.epi == EPI_ACT) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = act_apply(v[j], a.act);
+  } else if (a.resid && row < a.M) {
+    float r[32];
+    if (a.resid_fp32)
+      load_f32x32(static_cast<const float*>(a.resid) + static_cast<int64_t>(row) * a.ld_resid + n, r);
+    else
+      load_bf16x32(static_cast<const uint16_t*>(a.resid) + static_cast<int64_t>(row) * a.ld_resid + n, r);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] += r[j];
+  }
+}
+
+// Each epilogue warp owns two 2 KB staging buffers for 32 rows x 32 16-bit columns,
+// laid out like the 64-byte-swizzled TMA box: lane r's 16-byte piece j goes to
+// position j ^ ((r >> 1) & 3) of its 64-byte row (no bank conflicts).  Lane 0
+// stores the chunk at (x, y0) and recycles a buffer once the store issued two
+// chunks earlier has read it.
+__device__ __forceinline__ void stage_and_store(const GemmArgs& a, uint8_t* warp_staging, int& count, int lane,
+                                                const float (&v)[32], int x, int y0) {
+  uint8_t* buf = warp_staging + (count & 1) * 2048;
+  if (count >= 2) {
+    if (lane == 0) bulk_wait_group_read<1>();
+    __syncwarp();
+  }
+  uint32_t pk[16];
+  if (a.out_type == OUT_F16) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) pk[i] = pack_f16x2(v[2 * i], v[2 * i + 1]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+  }
+  const int sw = (lane >> 1) & 3;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ sw) << 4)) =
+        make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0 && y0 < a.M) {
+    tma_store_2d(&a.tmOut, buf, x, y0);
+    bulk_commit_group();
+  }
+  ++count;
+}
+
 // One 32-column chunk of one accumulator row: apply the epilogue and store.
 __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, const TileCoord& tc, int row, int n,
                                                float (&v)[32]) {
@@ -191,7 +251,8 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* staging = smem + STAGES * STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(staging + STAGING_BYTES);
   uint64_t* full_bar = bars;                       // [STAGES]
   uint64_t* empty_bar = bars + STAGES;             // [STAGES]
   uint64_t* acc_full = bars + 2 * STAGES;          // [NUM_ACC]
@@ -237,6 +298,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
     if (lane == 0) {
       tma_prefetch_desc(&a.tmA);
       for (int g = 0; g < a.G; ++g) tma_prefetch_desc(&a.tmB[g]);
+      if (a.tma_store) tma_prefetch_desc(&a.tmOut);
       // both operands are re-read by several CTAs at about the same time: default L2 policy
       const uint64_t pol_a = l2_policy_evict_normal();
       const uint64_t pol_b = pol_a;
@@ -326,6 +388,9 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
     const int col_half = (warp - 2) / 4;    // columns [col_half*BN/2, +BN/2) of each tile
     int acc = 0;
     uint32_t acc_phase = 0;
+    const bool tma_out = a.tma_store && (a.epi == EPI_ACT || a.epi == EPI_BIAS_RESID);
+    uint8_t* warp_staging = staging + (warp - 2) * 4096;
+    int store_count = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       if (*abort_flag) break;
       // the decision is made warp-uniform: tcgen05.ld below is a warp-collective instruction
@@ -355,10 +420,14 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
           tmem_ld_wait();
           const int cur = (c - c_begin) & 1;
           if (c + 1 < c_end) tmem_ld_32x32b_x32(t_row + (c + 1) * 32, r[cur ^ 1]);
-          if (row < a.M) {
-            float v[32];
+          float v[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[cur][j]);
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[cur][j]);
+          if (tma_out) {
+            epilogue_math(a, tc, row, n0 + c * 32, v);
+            const int x = (a.epi == EPI_ACT ? tc.g * static_cast<int>(a.out_col_per_group) : 0) + n0 + c * 32;
+            stage_and_store(a, warp_staging, store_count, lane, v, x, row - lane);
+          } else if (row < a.M) {
             epilogue_chunk(a, tc, row, n0 + c * 32, v);
           }
         }
@@ -369,6 +438,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
       if (++acc == NUM_ACC) { acc = 0; acc_phase ^= 1u; }
     }
+    if (lane == 0) bulk_wait_group_all();  // our output stores are complete before exit
   }
 
   tc_fence_before();
@@ -394,7 +464,7 @@ constexpr int P_STAGES = 6;
 constexpr int P_A_BYTES = BM * BK * 2;              // 16 KB per CTA
 constexpr int P_B_BYTES = (BN / 2) * BK * 2;        // 16 KB per CTA
 constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
-constexpr int P_SMEM_BYTES = 1024 + P_STAGES * P_STAGE_BYTES + 256;
+constexpr int P_SMEM_BYTES = 1024 + P_STAGES * P_STAGE_BYTES + STAGING_BYTES + 256;
 constexpr uint32_t P_IDESC_BF16 = idesc_bf16_f32(P_ROWS, BN, 0, 1);
 constexpr uint32_t P_IDESC_F16 = idesc_f16_f32(P_ROWS, BN, 0, 1);
 
@@ -404,7 +474,8 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sA = smem;
   uint8_t* sB = smem + P_STAGES * P_A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P_STAGES * P_STAGE_BYTES);
+  uint8_t* staging = smem + P_STAGES * P_STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(staging + STAGING_BYTES);
   uint64_t* full_bar = bars;                             // [P_STAGES], used in the leader
   uint64_t* empty_bar = bars + P_STAGES;                 // [P_STAGES], both CTAs
   uint64_t* acc_full = bars + 2 * P_STAGES;              // [NUM_ACC], both CTAs
@@ -453,6 +524,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
     if (lane == 0) {
       tma_prefetch_desc(&a.tmA);
       for (int g = 0; g < a.G; ++g) tma_prefetch_desc(&a.tmB[g]);
+      if (a.tma_store) tma_prefetch_desc(&a.tmOut);
       // both operands are re-read by several CTAs at about the same time: default L2 policy
       const uint64_t pol_a = l2_policy_evict_normal();
       const uint64_t pol_b = pol_a;
@@ -541,6 +613,9 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
     const uint32_t acc_empty0_leader = mapa_shared(smem_u32(&acc_empty[0]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
+    const bool tma_out = a.tma_store && (a.epi == EPI_ACT || a.epi == EPI_BIAS_RESID);
+    uint8_t* warp_staging = staging + (warp - 2) * 4096;
+    int store_count = 0;
     for (int tile = cid; tile < num_tiles; tile += nclusters) {
       if (*abort_flag) break;
       const bool ready = __all_sync(0xffffffffu,
@@ -569,10 +644,14 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
           tmem_ld_wait();
           const int cur = (c - c_begin) & 1;
           if (c + 1 < c_end) tmem_ld_32x32b_x32(t_row + (c + 1) * 32, r[cur ^ 1]);
-          if (row < a.M) {
-            float v[32];
+          float v[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[cur][j]);
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[cur][j]);
+          if (tma_out) {
+            epilogue_math(a, tc, row, n0 + c * 32, v);
+            const int x = (a.epi == EPI_ACT ? tc.g * static_cast<int>(a.out_col_per_group) : 0) + n0 + c * 32;
+            stage_and_store(a, warp_staging, store_count, lane, v, x, row - lane);
+          } else if (row < a.M) {
             epilogue_chunk(a, tc, row, n0 + c * 32, v);
           }
         }
@@ -583,6 +662,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
       if (lane == 0) mbar_arrive_cluster(acc_empty0_leader + static_cast<uint32_t>(acc) * 8u);
       if (++acc == NUM_ACC) { acc = 0; acc_phase ^= 1u; }
     }
+    if (lane == 0) bulk_wait_group_all();  // our output stores are complete before exit
   }
 
   __syncwarp();

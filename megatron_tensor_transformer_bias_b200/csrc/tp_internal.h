@@ -35,6 +35,7 @@ enum OutType : int { OUT_BF16 = 0, OUT_F32 = 1, OUT_F16 = 2 };
 enum Activation : int { ACT_NONE = 0, ACT_GELU = 1, ACT_RELU = 2 };
 
 struct __align__(64) GemmArgs {
+  CUtensorMap tmOut;                    // 16-bit output of EPI_ACT / EPI_BIAS_RESID, box {32, 32}, 64B swizzle
   CUtensorMap tmA;                      // A [M, Ktot] bf16 K-major, box {64, 128}, 128B swizzle
   CUtensorMap tmB[TP_MAX_SHARDS];       // B_g [Kg, N] bf16 N-major, box {64, 64}, 128B swizzle
   int M, N, Kg, G;
@@ -47,6 +48,7 @@ struct __align__(64) GemmArgs {
   int64_t out_col_per_group;            // EPI_ACT_BF16: column offset of group g in out
   int64_t out_group_stride;             // EPI_PARTIAL_F32: elements between partials
   int out_type;                         // OutType of EPI_ACT / EPI_BIAS_RESID
+  int tma_store;                        // 1: 16-bit EPI_ACT / EPI_BIAS_RESID output leaves through tmOut
   const void* bias_g[TP_MAX_SHARDS];    // bf16 [N] per group, or null
   const void* bias;                     // bf16 [N] or null (EPI_BIAS_RESID)
   const void* resid;                    // [M, N] or null
@@ -81,6 +83,9 @@ uint64_t wait_limit_ns();
 // 2-byte element tensor maps (bf16 or fp16), 128-byte swizzle, zero fill out of bounds.
 tp_status make_tmap_2d(CUtensorMap* map, const void* base, int f16, uint64_t inner, uint64_t outer,
                        uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+// Output map of the epilogue stores: box {32, 32} of a 2-byte type, 64-byte swizzle.
+tp_status make_tmap_out(CUtensorMap* map, void* base, int f16, uint64_t cols, uint64_t rows,
+                        uint64_t row_stride_bytes);
 
 // Kernel launchers.  All are asynchronous on `stream` and validate nothing:
 // the C-ABI layer has checked every argument before calling them.
