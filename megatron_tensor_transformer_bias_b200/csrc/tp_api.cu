@@ -169,11 +169,11 @@ static tp_status make_tmap_f16_3d(CUtensorMap* map, const void* base, uint64_t d
   return TP_OK;
 }
 
-tp_status make_tmap_attn(CUtensorMap* map, const void* base, int BH, int S, int d) {
-  // [B*H][S][d] fp16: inner d (box 64), then S (box 128), then heads (box 1).
+tp_status make_tmap_attn(CUtensorMap* map, const void* base, int BH, int S, int d, uint32_t box_rows) {
+  // [B*H][S][d] fp16: inner d (box 64), then S (box box_rows), then heads (box 1).
   return make_tmap_f16_3d(map, base, static_cast<uint64_t>(d), static_cast<uint64_t>(S),
                            static_cast<uint64_t>(BH), static_cast<uint64_t>(d) * 2,
-                           static_cast<uint64_t>(S) * d * 2, 64, 128);
+                           static_cast<uint64_t>(S) * d * 2, 64, box_rows);
 }
 
 }  // namespace tpb
@@ -409,9 +409,9 @@ tp_status attn_bf16(const void* X, int B, int S, int h, int H, int d, int t, con
   {
     AttnArgs a;
     memset(&a, 0, sizeof(a));
-    TP_TRY(make_tmap_attn(&a.tmQ, w.q, B * H, S, d));
-    TP_TRY(make_tmap_attn(&a.tmK, w.k, B * H, S, d));
-    TP_TRY(make_tmap_attn(&a.tmV, w.v, B * H, S, d));
+    TP_TRY(make_tmap_attn(&a.tmQ, w.q, B * H, S, d, 128));  // 128-query tiles
+    TP_TRY(make_tmap_attn(&a.tmK, w.k, B * H, S, d, 64));   // 64-key blocks
+    TP_TRY(make_tmap_attn(&a.tmV, w.v, B * H, S, d, 64));
     a.O = w.o; a.o_f16 = is_f16(Wo);
     a.B = B; a.S = S; a.H = H; a.d = d; a.causal = causal; a.head0 = 0;
     a.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(d));

@@ -6,12 +6,16 @@
 // All heads of all groups run in one launch; groups differ only in which
 // heads they own.
 //
-// One CTA per (128-query block, head, batch), 192 threads:
-//   warp 0      TMA: Q once, then K_j and V_j (128 keys each) into a 2-stage ring
-//   warp 1      TMEM allocation; one thread issues S_j = Q K_j^T and PV_j = P_j V_j
-//   warps 2..5  one query row per thread: row max and exp2 of S_j read from TMEM,
-//               P_j (fp16) written to shared memory in the MMA's swizzled layout,
-//               running max / sum, O kept in fp32 registers and rescaled per block.
+// One CTA per (128 queries, head, batch), two CTAs per SM, 192 threads:
+//   warp 0      TMA: Q once, then K_j (double-buffered) and V_j, 64 keys per block
+//   warp 1      TMEM allocation; one thread issues S_j = Q K_j^T into one of two
+//               TMEM score buffers, and O += P_j V_j into the TMEM output accumulator
+//   warps 2..5  one query row per thread: row max of S_j, P_j = exp2(s - m) in
+//               fp16 written to shared memory in the MMA's swizzled layout, row sum.
+// While the softmax warps work on S_j, the tensor core already computes S_{j+1}.
+// The running max is only moved (and O, l rescaled in place) when a row's max grows
+// by more than 2^8, so P stays <= 256 and the final O / l is unchanged; O never
+// leaves TMEM until the end.
 // Q, K, V are [B*H][S][d] fp16 (d = 128); O is written to [B*S, H*d] (bf16 or
 // fp16), the layout the row-parallel output projection reads.  Q, K and P are
 // fp16 because the scores' rounding error grows with |Q||K|: bf16 Q and K cost
@@ -23,18 +27,22 @@ namespace tpb {
 
 namespace {
 
-constexpr int BQ = 128;      // queries per CTA
-constexpr int BKV = 128;     // keys per block
-constexpr int D = 128;       // head dim
-constexpr int HALF_BYTES = 128 * 64 * 2;  // one [128 rows x 64 cols] bf16 swizzled box: 16 KB
-constexpr int TILE_BYTES = 2 * HALF_BYTES;  // [128 x 128] bf16: 32 KB
-constexpr int KV_STAGES = 2;
+constexpr int BQ = 128;                         // queries per CTA
+constexpr int BKV = 64;                         // keys per block
+constexpr int D = 128;                          // head dim
+constexpr int Q_HALF = BQ * 64 * 2;             // [128 rows x 64 d] fp16 swizzled box: 16 KB
+constexpr int Q_BYTES = 2 * Q_HALF;             // 32 KB
+constexpr int KV_HALF = BKV * 64 * 2;           // [64 rows x 64 d]: 8 KB
+constexpr int KV_BYTES = 2 * KV_HALF;           // 16 KB
+constexpr int P_BYTES = BQ * BKV * 2;           // [128 queries x 64 keys] fp16: 16 KB
 constexpr int THREADS = 192;
 constexpr int SOFTMAX_THREADS = 128;
-constexpr int SMEM_BYTES = 1024 + TILE_BYTES /*Q*/ + KV_STAGES * 2 * TILE_BYTES /*K,V*/ + TILE_BYTES /*P*/ + 256;
-constexpr uint32_t TMEM_COLS = 256;  // S: [0,128), PV: [128,256)
-constexpr uint32_t IDESC_S = idesc_f16_f32(BQ, BKV, 0, 0);    // Q K-major, K K-major (N = keys); fp16
-constexpr uint32_t IDESC_PV = idesc_f16_f32(BQ, D, 0, 1);     // P K-major, V N-major (N = d); fp16
+constexpr int SMEM_BYTES = 1024 + Q_BYTES + 2 * KV_BYTES /*K*/ + KV_BYTES /*V*/ + P_BYTES + 256;
+constexpr uint32_t TMEM_COLS = 256;             // S0 [0,64), S1 [64,128), O [128,256)
+constexpr uint32_t O_COL = 128;
+constexpr float RESCALE_LOG2 = 8.0f;            // move the running max only when it grows by > 2^8
+constexpr uint32_t IDESC_S = idesc_f16_f32(BQ, BKV, 0, 0);   // Q K-major, K K-major (N = keys)
+constexpr uint32_t IDESC_PV = idesc_f16_f32(BQ, D, 0, 1);    // P K-major, V N-major (N = d)
 
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, uint64_t* bar, int32_t x, int32_t y,
                                             int32_t z) {
@@ -45,23 +53,29 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, ui
       : "memory");
 }
 
-__global__ void __launch_bounds__(THREADS, 1) tp_attention_kernel(const __grid_constant__ AttnArgs a) {
+__device__ __forceinline__ bool visible(int kidx, int q, int S, int causal) {
+  return kidx < S && (!causal || kidx <= q);
+}
+
+__global__ void __launch_bounds__(THREADS, 2) tp_attention_kernel(const __grid_constant__ AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sQ = smem;
-  uint8_t* sK = sQ + TILE_BYTES;                       // [KV_STAGES] tiles
-  uint8_t* sV = sK + KV_STAGES * TILE_BYTES;           // [KV_STAGES] tiles
-  uint8_t* sP = sV + KV_STAGES * TILE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + TILE_BYTES);
+  uint8_t* sK = sQ + Q_BYTES;              // [2] blocks
+  uint8_t* sV = sK + 2 * KV_BYTES;
+  uint8_t* sP = sV + KV_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + P_BYTES);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;               // [KV_STAGES]
-  uint64_t* kv_empty = bars + 1 + KV_STAGES;  // [KV_STAGES]
-  uint64_t* s_full = bars + 1 + 2 * KV_STAGES;
-  uint64_t* p_full = s_full + 1;
-  uint64_t* pv_full = s_full + 2;
-  uint64_t* drain_bar = s_full + 3;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 4);
+  uint64_t* k_full = bars + 1;             // [2]
+  uint64_t* k_empty = bars + 3;            // [2]
+  uint64_t* v_full = bars + 5;
+  uint64_t* v_empty = bars + 6;
+  uint64_t* s_full = bars + 7;             // [2]
+  uint64_t* p_full = bars + 9;
+  uint64_t* pv_done = bars + 10;
+  uint64_t* drain_bar = bars + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32;
@@ -77,13 +91,15 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attention_kernel(const __grid_c
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < KV_STAGES; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&s_full[s], 1);
     }
-    mbar_init(s_full, 1);
+    mbar_init(v_full, 1);
+    mbar_init(v_empty, 1);
     mbar_init(p_full, SOFTMAX_THREADS);
-    mbar_init(pv_full, 1);
+    mbar_init(pv_done, 1);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -104,79 +120,88 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attention_kernel(const __grid_c
       tma_prefetch_desc(&a.tmQ);
       tma_prefetch_desc(&a.tmK);
       tma_prefetch_desc(&a.tmV);
-      mbar_arrive_expect_tx(q_full, TILE_BYTES);
+      mbar_arrive_expect_tx(q_full, Q_BYTES);
       tma_load_3d(sQ, &a.tmQ, q_full, 0, q0, bh);
-      tma_load_3d(sQ + HALF_BYTES, &a.tmQ, q_full, 64, q0, bh);
-      int issued = 0;
-      for (int j = 0; j < nkv; ++j) {
-        const int st = j % KV_STAGES;
-        const uint32_t ph = static_cast<uint32_t>(j / KV_STAGES) & 1u;
+      tma_load_3d(sQ + Q_HALF, &a.tmQ, q_full, 64, q0, bh);
+      int k_issued = 0, v_issued = 0;
+      bool ok = true;
+      // K runs up to two blocks ahead of V: K_j and K_{j+1} can be in flight while V_j
+      // waits for P_{j-1} V_{j-1} to release the single V buffer.
+      for (int j = 0; j <= nkv && ok; ++j) {
         if (*abort_flag) break;
-        if (!mbar_wait_bounded(&kv_empty[st], ph ^ 1u, a.wait_limit_ns, a.status, WAIT_SITE_ATTN)) {
-          *abort_flag = 1;
-          break;
+        if (j < nkv) {
+          const int ks = j & 1;
+          if (!mbar_wait_bounded(&k_empty[ks], ((j >> 1) & 1) ^ 1u, a.wait_limit_ns, a.status, WAIT_SITE_ATTN)) {
+            *abort_flag = 1; ok = false; break;
+          }
+          mbar_arrive_expect_tx(&k_full[ks], KV_BYTES);
+          tma_load_3d(sK + ks * KV_BYTES, &a.tmK, &k_full[ks], 0, j * BKV, bh);
+          tma_load_3d(sK + ks * KV_BYTES + KV_HALF, &a.tmK, &k_full[ks], 64, j * BKV, bh);
+          ++k_issued;
         }
-        mbar_arrive_expect_tx(&kv_full[st], 2 * TILE_BYTES);
-        uint8_t* k_dst = sK + st * TILE_BYTES;
-        uint8_t* v_dst = sV + st * TILE_BYTES;
-        tma_load_3d(k_dst, &a.tmK, &kv_full[st], 0, j * BKV, bh);
-        tma_load_3d(k_dst + HALF_BYTES, &a.tmK, &kv_full[st], 64, j * BKV, bh);
-        tma_load_3d(v_dst, &a.tmV, &kv_full[st], 0, j * BKV, bh);
-        tma_load_3d(v_dst + HALF_BYTES, &a.tmV, &kv_full[st], 64, j * BKV, bh);
-        ++issued;
+        if (j >= 1) {
+          const int jv = j - 1;
+          if (!mbar_wait_bounded(v_empty, (jv & 1) ^ 1u, a.wait_limit_ns, a.status, WAIT_SITE_ATTN)) {
+            *abort_flag = 1; ok = false; break;
+          }
+          mbar_arrive_expect_tx(v_full, KV_BYTES);
+          tma_load_3d(sV, &a.tmV, v_full, 0, jv * BKV, bh);
+          tma_load_3d(sV + KV_HALF, &a.tmV, v_full, 64, jv * BKV, bh);
+          ++v_issued;
+        }
       }
       // wait for our own copies in flight
       mbar_wait_bounded(q_full, 0, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
-      for (int j = issued - KV_STAGES > 0 ? issued - KV_STAGES : 0; j < issued; ++j)
-        mbar_wait_bounded(&kv_full[j % KV_STAGES], static_cast<uint32_t>(j / KV_STAGES) & 1u, a.wait_limit_ns,
-                          a.status, WAIT_SITE_ATTN);
+      for (int j = k_issued - 2 > 0 ? k_issued - 2 : 0; j < k_issued; ++j)
+        mbar_wait_bounded(&k_full[j & 1], (j >> 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
+      if (v_issued > 0) mbar_wait_bounded(v_full, (v_issued - 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t qa = smem_u32(sQ);
       const uint32_t pa = smem_u32(sP);
-      const uint32_t t_s = tmem_base;
-      const uint32_t t_pv = tmem_base + 128;
+      const uint32_t va = smem_u32(sV);
+      const uint32_t t_o = tmem_base + O_COL;
       bool ok = mbar_wait_bounded(q_full, 0, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
       if (!ok) *abort_flag = 1;
       for (int j = 0; j <= nkv && ok; ++j) {
         if (j < nkv) {
-          const int st = j % KV_STAGES;
-          if (!mbar_wait_bounded(&kv_full[st], static_cast<uint32_t>(j / KV_STAGES) & 1u, a.wait_limit_ns,
-                                 a.status, WAIT_SITE_ATTN)) {
+          const int ks = j & 1;
+          if (!mbar_wait_bounded(&k_full[ks], (j >> 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN)) {
             *abort_flag = 1; ok = false; break;
           }
-        }
-        if (j > 0) {
-          // softmax has read S_{j-1} and PV_{j-2} and written P_{j-1}
-          if (!mbar_wait_bounded(p_full, static_cast<uint32_t>(j - 1) & 1u, a.wait_limit_ns, a.status,
-                                 WAIT_SITE_ATTN)) {
-            *abort_flag = 1; ok = false; break;
-          }
-        }
-        tc_fence_after();
-        if (j < nkv) {
-          const uint32_t ka = smem_u32(sK + (j % KV_STAGES) * TILE_BYTES);
+          // score buffer ks held S_{j-2}; the softmax released it with p_full(j-2), which this
+          // thread already waited for before issuing P_{j-2} V_{j-2} (waiting again here could
+          // see the barrier two phases on and stall)
+          tc_fence_after();
+          const uint32_t ka = smem_u32(sK + ks * KV_BYTES);
+          const uint32_t t_s = tmem_base + static_cast<uint32_t>(ks * BKV);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-            mma_bf16_ss(t_s, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), IDESC_S,
+            const uint32_t qoff = (kk >> 2) * Q_HALF + (kk & 3) * 32;
+            const uint32_t koff = (kk >> 2) * KV_HALF + (kk & 3) * 32;
+            mma_bf16_ss(t_s, smem_desc_sw128(qa + qoff, 16, 1024), smem_desc_sw128(ka + koff, 16, 1024), IDESC_S,
                         kk > 0 ? 1u : 0u);
           }
-          mma_commit(s_full);
+          mma_commit(&s_full[ks]);
+          mma_commit(&k_empty[ks]);
         }
-        if (j > 0) {
+        if (j >= 1) {
           const int jp = j - 1;
-          const uint32_t va = smem_u32(sV + (jp % KV_STAGES) * TILE_BYTES);
+          // P_{jp} written (and O rescaled) by the softmax, V_{jp} loaded
+          if (!mbar_wait_bounded(p_full, jp & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN) ||
+              !mbar_wait_bounded(v_full, jp & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN)) {
+            *abort_flag = 1; ok = false; break;
+          }
+          tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < BKV / 16; ++kk) {
-            const uint32_t poff = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-            mma_bf16_ss(t_pv, smem_desc_sw128(pa + poff, 16, 1024),
-                        smem_desc_sw128(va + kk * 16 * 128, HALF_BYTES, 1024), IDESC_PV, kk > 0 ? 1u : 0u);
+            mma_bf16_ss(t_o, smem_desc_sw128(pa + kk * 32, 16, 1024),
+                        smem_desc_sw128(va + kk * 16 * 128, KV_HALF, 1024), IDESC_PV, (jp > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(pv_full);
-          mma_commit(&kv_empty[jp % KV_STAGES]);
+          mma_commit(pv_done);
+          mma_commit(v_empty);
         }
       }
       mma_commit(drain_bar);
@@ -188,132 +213,113 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attention_kernel(const __grid_c
     const int r = sub * 32 + lane;      // query row within the block
     const int q = q0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
-    const uint32_t t_s = tmem_base + lane_off;
-    const uint32_t t_pv = tmem_base + 128 + lane_off;
+    const uint32_t t_o = tmem_base + O_COL + lane_off;
     const float sl2 = a.scale_log2;
-    float o[D];
-#pragma unroll
-    for (int i = 0; i < D; ++i) o[i] = 0.f;
-    float m_run = -INFINITY;   // running max of scaled scores (log2 units)
+    float m_ref = -INFINITY;   // reference max of the scaled scores (log2 units)
     float l_run = 0.f;
-    float alpha_pending = 0.f; // rescale factor to apply together with PV_{j-1}
     bool ok = true;
     uint8_t* p_row = sP + r * 128;
     const int rsw = r & 7;
     for (int j = 0; j < nkv && ok; ++j) {
-      // waits are made warp-uniform: tcgen05.ld is a warp-collective instruction
-      if (!__all_sync(0xffffffffu, mbar_wait_bounded(s_full, static_cast<uint32_t>(j) & 1u, a.wait_limit_ns,
-                                                     a.status, WAIT_SITE_ATTN))) {
+      const int ks = j & 1;
+      // waits are made warp-uniform: tcgen05.ld/st are warp-collective instructions
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&s_full[ks], (j >> 1) & 1, a.wait_limit_ns, a.status,
+                                                     WAIT_SITE_ATTN))) {
         *abort_flag = 1; ok = false; break;
       }
       tc_fence_after();
+      const uint32_t t_s = tmem_base + lane_off + static_cast<uint32_t>(ks * BKV);
       const int k0 = j * BKV;
-      // pass 1: row max over visible keys
+      uint32_t sr[2][32];
+      tmem_ld_32x32b_x32(t_s, sr[0]);
+      tmem_ld_32x32b_x32(t_s + 32, sr[1]);
+      tmem_ld_wait();
       float mx = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < BKV / 32; ++c) {
-        uint32_t sr[32];
-        tmem_ld_32x32b_x32(t_s + c * 32, sr);
-        tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int kidx = k0 + c * 32 + i;
-          const bool vis = kidx < a.S && (!a.causal || kidx <= q);
-          if (vis) mx = fmaxf(mx, __uint_as_float(sr[i]) * sl2);
-        }
-      }
-      const float m_new = fmaxf(m_run, mx);
-      const float m_use = m_new == -INFINITY ? 0.f : m_new;
-      const float alpha = exp2f(m_run - m_use);  // 0 on the first block
-      // before overwriting sP: PV_{j-1} must be complete; fold it into O
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (visible(k0 + c * 32 + i, q, a.S, a.causal)) mx = fmaxf(mx, __uint_as_float(sr[c][i]) * sl2);
+      // the reference max moves only when the row max exceeds it by more than 2^8
+      const bool move = mx > m_ref + RESCALE_LOG2;
+      const float m_new = move ? mx : m_ref;
+      // P_{j-1} V_{j-1} must be done before P_j overwrites the P buffer and before O is rescaled
       if (j > 0) {
-        if (!__all_sync(0xffffffffu, mbar_wait_bounded(pv_full, static_cast<uint32_t>(j - 1) & 1u,
-                                                       a.wait_limit_ns, a.status, WAIT_SITE_ATTN))) {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(pv_done, (j - 1) & 1, a.wait_limit_ns, a.status,
+                                                       WAIT_SITE_ATTN))) {
           *abort_flag = 1; ok = false; break;
         }
         tc_fence_after();
+        if (__any_sync(0xffffffffu, move)) {
+          const float alpha = move ? exp2f(m_ref - m_new) : 1.0f;
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld_32x32b_x32(t_o + c * 32, o);
+            tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t pr[32];
-          tmem_ld_32x32b_x32(t_pv + c * 32, pr);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[c * 32 + i] = o[c * 32 + i] * alpha_pending + __uint_as_float(pr[i]);
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st_32x32b_x32(t_o + c * 32, o);
+          }
+          tmem_st_wait();
+          l_run *= alpha;
         }
       }
-      // pass 2: P = exp2(s - m), rounded to fp16, written in the 128B-swizzled K-major layout
+      const float m_use = m_new == -INFINITY ? 0.f : m_new;
+      m_ref = m_new;
+      // P = exp2(s - m) in fp16, written in the 128B-swizzled K-major layout (one 128-byte row per query)
       float lsum = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < BKV / 32; ++c) {
-        uint32_t sr[32];
-        tmem_ld_32x32b_x32(t_s + c * 32, sr);
-        tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          float pv2[2];
+          float e2[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int kidx = k0 + c * 32 + 2 * i + e;
-            const bool vis = kidx < a.S && (!a.causal || kidx <= q);
-            pv2[e] = vis ? exp2f(__uint_as_float(sr[2 * i + e]) * sl2 - m_use) : 0.f;
+            e2[e] = visible(kidx, q, a.S, a.causal) ? exp2f(__uint_as_float(sr[c][2 * i + e]) * sl2 - m_use) : 0.f;
           }
-          __half2 hb = __floats2half2_rn(pv2[0], pv2[1]);
+          __half2 hb = __floats2half2_rn(e2[0], e2[1]);
           lsum += __low2float(hb) + __high2float(hb);
           pk[i] = *reinterpret_cast<uint32_t*>(&hb);
         }
-        // 32 keys = 4 chunks of 8; key block (c*32)/64, chunk within the 128B row
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int key = c * 32 + u * 8;
-          const int blk = key >> 6;
-          const int chunk = (key & 63) >> 3;
-          uint4* dst = reinterpret_cast<uint4*>(p_row + blk * HALF_BYTES + ((chunk ^ rsw) << 4));
-          *dst = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+          const int chunk = c * 4 + u;   // 8 keys per 16-byte chunk
+          *reinterpret_cast<uint4*>(p_row + ((chunk ^ rsw) << 4)) =
+              make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         }
       }
-      l_run = l_run * alpha + lsum;
-      m_run = m_new;
-      alpha_pending = alpha;
-      // publish P_j to the tensor core (async proxy) and release S_j
+      l_run += lsum;
+      // publish P_j to the tensor core (async proxy); S_j and O are released with it
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(p_full);
     }
     if (ok && nkv > 0) {
-      if (__all_sync(0xffffffffu, mbar_wait_bounded(pv_full, static_cast<uint32_t>(nkv - 1) & 1u,
-                                                    a.wait_limit_ns, a.status, WAIT_SITE_ATTN))) {
+      if (__all_sync(0xffffffffu, mbar_wait_bounded(pv_done, (nkv - 1) & 1, a.wait_limit_ns, a.status,
+                                                    WAIT_SITE_ATTN))) {
         tc_fence_after();
-#pragma unroll
+        const float inv = 1.f / l_run;
+        uint16_t* dst = static_cast<uint16_t*>(a.O) + (static_cast<int64_t>(b) * a.S + q) * (a.H * D) + head * D;
+#pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
-          uint32_t pr[32];
-          tmem_ld_32x32b_x32(t_pv + c * 32, pr);
+          uint32_t o[32];
+          tmem_ld_32x32b_x32(t_o + c * 32, o);
           tmem_ld_wait();
+          if (q < a.S) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[c * 32 + i] = o[c * 32 + i] * alpha_pending + __uint_as_float(pr[i]);
-        }
-        if (q < a.S) {
-          const float inv = 1.f / l_run;
-          uint16_t* dst = static_cast<uint16_t*>(a.O) + (static_cast<int64_t>(b) * a.S + q) * (a.H * D) + head * D;
-          if (a.o_f16) {
+            for (int u = 0; u < 4; ++u) {
+              uint4 w;
+              uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
-            for (int c = 0; c < D / 8; ++c) {
-              uint4 u;
-              u.x = pack_f16x2(o[c * 8 + 0] * inv, o[c * 8 + 1] * inv);
-              u.y = pack_f16x2(o[c * 8 + 2] * inv, o[c * 8 + 3] * inv);
-              u.z = pack_f16x2(o[c * 8 + 4] * inv, o[c * 8 + 5] * inv);
-              u.w = pack_f16x2(o[c * 8 + 6] * inv, o[c * 8 + 7] * inv);
-              reinterpret_cast<uint4*>(dst)[c] = u;
-            }
-          } else {
-#pragma unroll
-            for (int c = 0; c < D / 8; ++c) {
-              uint4 u;
-              u.x = pack_bf16x2(o[c * 8 + 0] * inv, o[c * 8 + 1] * inv);
-              u.y = pack_bf16x2(o[c * 8 + 2] * inv, o[c * 8 + 3] * inv);
-              u.z = pack_bf16x2(o[c * 8 + 4] * inv, o[c * 8 + 5] * inv);
-              u.w = pack_bf16x2(o[c * 8 + 6] * inv, o[c * 8 + 7] * inv);
-              reinterpret_cast<uint4*>(dst)[c] = u;
+              for (int e = 0; e < 4; ++e) {
+                const float lo = __uint_as_float(o[u * 8 + 2 * e]) * inv;
+                const float hi = __uint_as_float(o[u * 8 + 2 * e + 1]) * inv;
+                wp[e] = a.o_f16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
+              }
+              reinterpret_cast<uint4*>(dst + c * 32)[u] = w;
             }
           }
         }

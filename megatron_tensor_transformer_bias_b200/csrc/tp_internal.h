@@ -63,8 +63,8 @@ struct __align__(64) GemmArgs {
 
 struct AttnArgs {
   CUtensorMap tmQ;   // Q [B*H][S][d] fp16, box {64, 128, 1}, 128B swizzle
-  CUtensorMap tmK;   // K [B*H][S][d] fp16
-  CUtensorMap tmV;   // V [B*H][S][d] fp16
+  CUtensorMap tmK;   // K [B*H][S][d] fp16, box {64, 64, 1}
+  CUtensorMap tmV;   // V [B*H][S][d] fp16, box {64, 64, 1}
   void* O;           // O [B*S, H*d] (head-major columns), bf16 or fp16
   int o_f16;
   int B, S, H, d, causal;
