@@ -5,6 +5,7 @@
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <string>
 #include <vector>
@@ -84,6 +85,15 @@ uint32_t* device_status_ptr() {
 }
 
 uint64_t wait_limit_ns() { return g_wait_limit_ns.load(); }
+
+bool pdl_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("TPB_PDL");
+    v = (e && e[0] == '0') ? 0 : 1;
+  }
+  return v == 1;
+}
 
 tp_status set_error(tp_status s, const char* msg) {
   t_last_error = msg;

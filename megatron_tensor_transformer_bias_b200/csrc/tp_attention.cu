@@ -113,6 +113,7 @@ __global__ void __launch_bounds__(THREADS, 2) tp_attention_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // Q, K, V come from the preceding projection kernel
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -329,6 +330,7 @@ __global__ void __launch_bounds__(THREADS, 2) tp_attention_kernel(const __grid_c
     }
   }
 
+  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -354,8 +356,8 @@ tp_status launch_attention(const AttnArgs& a, cudaStream_t stream) {
   if (nqb == 0 || a.B == 0) return TP_OK;
   dim3 grid(nqb, a.H - a.head0, a.B);
   trace_before(stream);
-  tp_attention_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(a);
-  if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
+  const tp_status st = launch_ex(tp_attention_kernel, grid, dim3(THREADS), SMEM_BYTES, stream, 1, a);
+  if (st != TP_OK) return st;
   trace_after(stream, "attention");
   return TP_OK;
 }

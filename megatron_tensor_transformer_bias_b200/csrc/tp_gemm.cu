@@ -292,6 +292,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_base_slot;
+  pdl_wait();  // the previous kernel's outputs (our operands, our workspace) are complete
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -441,6 +442,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
     if (lane == 0) bulk_wait_group_all();  // our output stores are complete before exit
   }
 
+  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -518,6 +520,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
   cluster_sync_all();  // barriers of both CTAs initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_base_slot;
+  pdl_wait();  // the previous kernel's outputs (our operands, our workspace) are complete
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -665,6 +668,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
     if (lane == 0) bulk_wait_group_all();  // our output stores are complete before exit
   }
 
+  pdl_launch_dependents();
   __syncwarp();
   tc_fence_before();
   cluster_sync_all();  // the leader's MMAs and the remote arrives are done in both CTAs
@@ -721,21 +725,9 @@ static tp_status launch_gemm_pair(const GemmArgs& a, cudaStream_t stream, const 
   const long long tiles = 1LL * m_tiles * n_tiles * (a.concat ? 1 : a.G);
   if (tiles <= 0) return TP_OK;
   const int nclusters = static_cast<int>(tiles < nclusters_max ? tiles : nclusters_max);
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3(2 * nclusters, 1, 1);
-  cfg.blockDim = dim3(THREADS, 1, 1);
-  cfg.dynamicSmemBytes = P_SMEM_BYTES;
-  cfg.stream = stream;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   trace_before(stream);
-  if (cudaLaunchKernelEx(&cfg, tp_gemm_pair_kernel, a) != cudaSuccess) return TP_ERR_CUDA;
-  if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
+  const tp_status st = launch_ex(tp_gemm_pair_kernel, dim3(2 * nclusters), dim3(THREADS), P_SMEM_BYTES, stream, 2, a);
+  if (st != TP_OK) return st;
   trace_after(stream, name);
   return TP_OK;
 }
@@ -757,8 +749,8 @@ tp_status launch_gemm(const GemmArgs& a, cudaStream_t stream, const char* name) 
   if (tiles <= 0) return TP_OK;
   const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
   trace_before(stream);
-  tp_gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(a);
-  if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
+  const tp_status st = launch_ex(tp_gemm_kernel, dim3(grid), dim3(THREADS), SMEM_BYTES, stream, 1, a);
+  if (st != TP_OK) return st;
   trace_after(stream, name);
   return TP_OK;
 }

@@ -102,6 +102,38 @@ tp_status launch_ffn_fp32(const float* X, int64_t M, int64_t h, int64_t f, int t
 tp_status launch_selftest_wait(uint64_t limit_ns, cudaStream_t stream);
 tp_status launch_act(const float* x, float* y, int64_t n, int act, cudaStream_t stream);
 
+// Launch `kern` on `stream` with programmatic dependent launch (the kernel waits for
+// its predecessor with griddepcontrol.wait before touching global memory) and an
+// optional cluster size.  TPB_PDL=0 turns the attribute off.
+bool pdl_enabled();
+template <typename... KArgs, typename... Args>
+tp_status launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, int cluster_x,
+                    Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  if (cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...) != cudaSuccess) return TP_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}
+
 // Record `msg` as the calling thread's tp_last_error() and return `s`.
 tp_status set_error(tp_status s, const char* msg);
 

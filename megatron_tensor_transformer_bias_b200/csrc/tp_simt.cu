@@ -30,6 +30,7 @@ __global__ void __launch_bounds__(256) reduce_partials_kernel(const float* __res
                                                               void* __restrict__ out) {
   const int64_t nvec = MH / 4;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  pdl_wait();
   for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < nvec; v += stride) {
     const int64_t e = v * 4;
     // fixed shard order 0..t-1
@@ -55,6 +56,7 @@ __global__ void __launch_bounds__(256) reduce_partials_kernel(const float* __res
       *reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + e) = o;
     }
   }
+  pdl_launch_dependents();
 }
 
 // ---------------------------------------------------------------- layernorm
@@ -83,6 +85,7 @@ __global__ void __launch_bounds__(LN_THREADS) layernorm_kernel(const void* __res
   const int64_t r = blockIdx.x;
   const int64_t n8 = h / 8;
   float s = 0.f;
+  pdl_wait();
   for (int64_t v = threadIdx.x; v < n8; v += LN_THREADS) {
     float f[8];
     if (IN_F32) {
@@ -135,6 +138,7 @@ __global__ void __launch_bounds__(LN_THREADS) layernorm_kernel(const void* __res
     }
     reinterpret_cast<uint4*>(y + r * h)[v] = u;
   }
+  pdl_launch_dependents();
 }
 
 // ---------------------------------------------------------------- exact fp32 FFN
@@ -212,9 +216,13 @@ tp_status launch_reduce_partials(const float* P, int t, int64_t M, int64_t h, co
   const int g = static_cast<int>(blocks);
   const int key = (out_fp32 ? 4 : 0) | (resid_fp32 ? 2 : 0) | (bias_fp32 ? 1 : 0);
   trace_before(stream);
+  tp_status st = TP_OK;
   switch (key) {
-#define TP_REDUCE_CASE(K, O, R, B) \
-    case K: reduce_partials_kernel<O, R, B><<<g, 256, 0, stream>>>(P, t, M * h, bias, h, resid, out); break;
+#define TP_REDUCE_CASE(K, O, R, B)                                                                              \
+    case K:                                                                                                    \
+      st = launch_ex(reduce_partials_kernel<O, R, B>, dim3(g), dim3(256), 0, stream, 1, P, t, M * h, bias, h, \
+                     resid, out);                                                                              \
+      break;
     TP_REDUCE_CASE(0, false, false, false)
     TP_REDUCE_CASE(1, false, false, true)
     TP_REDUCE_CASE(2, false, true, false)
@@ -225,7 +233,7 @@ tp_status launch_reduce_partials(const float* P, int t, int64_t M, int64_t h, co
     TP_REDUCE_CASE(7, true, true, true)
 #undef TP_REDUCE_CASE
   }
-  if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
+  if (st != TP_OK) return st;
   trace_after(stream, "reduce_partials");
   return TP_OK;
 }
@@ -248,10 +256,10 @@ tp_status launch_layernorm(const void* x, int in_fp32, const void* g, const void
     attr_set[dev][key] = 1;
   }
   trace_before(stream);
-  kern<<<static_cast<unsigned>(M), LN_THREADS, smem, stream>>>(x, static_cast<const uint16_t*>(g),
-                                                               static_cast<const uint16_t*>(b), h, eps,
-                                                               static_cast<uint16_t*>(y));
-  if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
+  const tp_status st = launch_ex(kern, dim3(static_cast<unsigned>(M)), dim3(LN_THREADS), smem, stream, 1, x,
+                                 static_cast<const uint16_t*>(g), static_cast<const uint16_t*>(b), h, eps,
+                                 static_cast<uint16_t*>(y));
+  if (st != TP_OK) return st;
   trace_after(stream, "layernorm");
   return TP_OK;
 }
