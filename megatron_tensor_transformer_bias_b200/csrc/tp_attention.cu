@@ -53,8 +53,35 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, ui
       : "memory");
 }
 
-__device__ __forceinline__ bool visible(int kidx, int q, int S, int causal) {
-  return kidx < S && (!causal || kidx <= q);
+// 2^x with the MUFU instruction (relative error ~2^-22; inputs below -126 give +0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// (d0, d1) = (a0 * b + c, a1 * b + c) as one packed fp32x2 instruction
+__device__ __forceinline__ void fma2_bc(float& d0, float& d1, float a0, float a1, float b, float c) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\tmov.b64 rc, {%5, %5};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+
+// (s0, s1) += (a0, a1) as one packed fp32x2 instruction
+__device__ __forceinline__ void add2_acc(float& s0, float& s1, float a0, float a1) {
+  asm("{\n\t.reg .b64 ra, rs;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rs, {%0, %1};\n\t"
+      "add.rn.f32x2 rs, rs, ra;\n\tmov.b64 {%0, %1}, rs;\n\t}"
+      : "+f"(s0), "+f"(s1)
+      : "f"(a0), "f"(a1));
 }
 
 __global__ void __launch_bounds__(THREADS, 2) tp_attention_kernel(const __grid_constant__ AttnArgs a) {
@@ -235,13 +262,29 @@ __global__ void __launch_bounds__(THREADS, 2) tp_attention_kernel(const __grid_c
       tmem_ld_32x32b_x32(t_s, sr[0]);
       tmem_ld_32x32b_x32(t_s + 32, sr[1]);
       tmem_ld_wait();
-      float mx = -INFINITY;
+      // Keys k0 + i with i <= lim are visible to this row (causal, and inside the
+      // sequence); a block every row sees whole takes the mask-free path.
+      const int lim = min(a.causal ? q - k0 : BKV - 1, a.S - 1 - k0);
+      const bool whole = k0 + BKV <= a.S && (!a.causal || k0 + BKV - 1 <= q0);
+      if (!whole) {
 #pragma unroll
-      for (int c = 0; c < 2; ++c)
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (visible(k0 + c * 32 + i, q, a.S, a.causal)) mx = fmaxf(mx, __uint_as_float(sr[c][i]) * sl2);
-      // the reference max moves only when the row max exceeds it by more than 2^8
+          for (int i = 0; i < 32; ++i)
+            if (c * 32 + i > lim) sr[c][i] = __float_as_uint(-INFINITY);
+      }
+      // row max of the raw scores, then scaled (the scale is positive)
+      float mx;
+      {
+        float m4[4] = {__uint_as_float(sr[0][0]), __uint_as_float(sr[0][1]), __uint_as_float(sr[1][0]),
+                       __uint_as_float(sr[1][1])};
+#pragma unroll
+        for (int i = 2; i < 32; i += 2) {
+          m4[0] = max3f(m4[0], __uint_as_float(sr[0][i]), __uint_as_float(sr[0][i + 1]));
+          m4[1] = max3f(m4[1], __uint_as_float(sr[1][i]), __uint_as_float(sr[1][i + 1]));
+        }
+        mx = max3f(m4[0], m4[1], fmaxf(m4[2], m4[3])) * sl2;
+      }
       const bool move = mx > m_ref + RESCALE_LOG2;
       const float m_new = move ? mx : m_ref;
       // P_{j-1} V_{j-1} must be done before P_j overwrites the P buffer and before O is rescaled
@@ -268,22 +311,21 @@ __global__ void __launch_bounds__(THREADS, 2) tp_attention_kernel(const __grid_c
       }
       const float m_use = m_new == -INFINITY ? 0.f : m_new;
       m_ref = m_new;
-      // P = exp2(s - m) in fp16, written in the 128B-swizzled K-major layout (one 128-byte row per query)
-      float lsum = 0.f;
+      // P = exp2(s * scale - m) in fp16, written in the 128B-swizzled K-major layout (one
+      // 128-byte row per query); masked scores are -inf and give 0.  The row sum is taken
+      // over the fp32 values.
+      float ls0 = 0.f, ls1 = 0.f;
+      const float neg_m = -m_use;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          float e2[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int kidx = k0 + c * 32 + 2 * i + e;
-            e2[e] = visible(kidx, q, a.S, a.causal) ? exp2f(__uint_as_float(sr[c][2 * i + e]) * sl2 - m_use) : 0.f;
-          }
-          __half2 hb = __floats2half2_rn(e2[0], e2[1]);
-          lsum += __low2float(hb) + __high2float(hb);
-          pk[i] = *reinterpret_cast<uint32_t*>(&hb);
+          float x0, x1;
+          fma2_bc(x0, x1, __uint_as_float(sr[c][2 * i]), __uint_as_float(sr[c][2 * i + 1]), sl2, neg_m);
+          const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
+          add2_acc(ls0, ls1, e0, e1);
+          pk[i] = pack_f16x2(e0, e1);
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -292,6 +334,7 @@ __global__ void __launch_bounds__(THREADS, 2) tp_attention_kernel(const __grid_c
               make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         }
       }
+      const float lsum = ls0 + ls1;
       l_run += lsum;
       // publish P_j to the tensor core (async proxy); S_j and O are released with it
       fence_proxy_async_smem();
