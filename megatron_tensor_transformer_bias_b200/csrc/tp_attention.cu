@@ -11,8 +11,11 @@
 //   warp 1      TMEM allocation; one thread issues S_j = Q K_j^T into one of two
 //               TMEM score buffers, and O += P_j V_j into the TMEM output accumulator
 //   warps 2..5  one query row per thread: row max of S_j, P_j = exp2(s - m) in
-//               fp16 written to shared memory in the MMA's swizzled layout, row sum.
-// While the softmax warps work on S_j, the tensor core already computes S_{j+1}.
+//               fp16 written back over S_j in tensor memory, row sum.
+// O += P_j V_j reads P_j from tensor memory (A operand in TMEM) and V_j from shared
+// memory, so P is double-buffered with the scores and the softmax of block j does not
+// wait for P_{j-1} V_{j-1}.  While the softmax warps work on S_j, the tensor core
+// already computes S_{j+1}.
 // The running max is only moved (and O, l rescaled in place) when a row's max grows
 // by more than 2^8, so P stays <= 256 and the final O / l is unchanged; O never
 // leaves TMEM until the end.
@@ -34,15 +37,26 @@ constexpr int Q_HALF = BQ * 64 * 2;             // [128 rows x 64 d] fp16 swizzl
 constexpr int Q_BYTES = 2 * Q_HALF;             // 32 KB
 constexpr int KV_HALF = BKV * 64 * 2;           // [64 rows x 64 d]: 8 KB
 constexpr int KV_BYTES = 2 * KV_HALF;           // 16 KB
-constexpr int P_BYTES = BQ * BKV * 2;           // [128 queries x 64 keys] fp16: 16 KB
 constexpr int THREADS = 192;
 constexpr int SOFTMAX_THREADS = 128;
-constexpr int SMEM_BYTES = 1024 + Q_BYTES + 2 * KV_BYTES /*K*/ + KV_BYTES /*V*/ + P_BYTES + 256;
-constexpr uint32_t TMEM_COLS = 256;             // S0 [0,64), S1 [64,128), O [128,256)
+constexpr int SMEM_BYTES = 1024 + Q_BYTES + 2 * KV_BYTES /*K*/ + KV_BYTES /*V*/ + 256;
+constexpr uint32_t TMEM_COLS = 256;             // S0 [0,64), S1 [64,128), O [128,256); P_j over S_j
 constexpr uint32_t O_COL = 128;
 constexpr float RESCALE_LOG2 = 8.0f;            // move the running max only when it grows by > 2^8
 constexpr uint32_t IDESC_S = idesc_f16_f32(BQ, BKV, 0, 0);   // Q K-major, K K-major (N = keys)
-constexpr uint32_t IDESC_PV = idesc_f16_f32(BQ, D, 0, 1);    // P K-major, V N-major (N = d)
+constexpr uint32_t IDESC_PV = idesc_f16_f32(BQ, D, 0, 1);    // P (TMEM, K-major), V N-major (N = d)
+
+// D[tmem] (+)= A[tmem] * B[smem desc]: fp16 A read from tensor memory, lane = row,
+// two 16-bit K elements per 32-bit column (the lower K index in the low half).
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, uint64_t* bar, int32_t x, int32_t y,
                                             int32_t z) {
@@ -91,18 +105,21 @@ __global__ void __launch_bounds__(THREADS, 2) tp_attention_kernel(const __grid_c
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + Q_BYTES;              // [2] blocks
   uint8_t* sV = sK + 2 * KV_BYTES;
-  uint8_t* sP = sV + KV_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + P_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + KV_BYTES);
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;             // [2]
   uint64_t* k_empty = bars + 3;            // [2]
   uint64_t* v_full = bars + 5;
   uint64_t* v_empty = bars + 6;
   uint64_t* s_full = bars + 7;             // [2]
+  // [2], by block parity: a softmax warp can finish block j+1 while another is still on
+  // block j (P_j no longer waits for P_{j-1} V_{j-1}), so the two blocks' arrivals must
+  // not meet on one barrier.  It cannot get two blocks ahead: S_{j+2} is issued only
+  // after P_j V_j, which needs every arrival of block j.
   uint64_t* p_full = bars + 9;
-  uint64_t* pv_done = bars + 10;
-  uint64_t* drain_bar = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* pv_done = bars + 11;
+  uint64_t* drain_bar = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32;
@@ -125,7 +142,8 @@ __global__ void __launch_bounds__(THREADS, 2) tp_attention_kernel(const __grid_c
     }
     mbar_init(v_full, 1);
     mbar_init(v_empty, 1);
-    mbar_init(p_full, SOFTMAX_THREADS);
+    mbar_init(&p_full[0], SOFTMAX_THREADS);
+    mbar_init(&p_full[1], SOFTMAX_THREADS);
     mbar_init(pv_done, 1);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -188,7 +206,6 @@ __global__ void __launch_bounds__(THREADS, 2) tp_attention_kernel(const __grid_c
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t qa = smem_u32(sQ);
-      const uint32_t pa = smem_u32(sP);
       const uint32_t va = smem_u32(sV);
       const uint32_t t_o = tmem_base + O_COL;
       bool ok = mbar_wait_bounded(q_full, 0, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
@@ -217,16 +234,17 @@ __global__ void __launch_bounds__(THREADS, 2) tp_attention_kernel(const __grid_c
         }
         if (j >= 1) {
           const int jp = j - 1;
-          // P_{jp} written (and O rescaled) by the softmax, V_{jp} loaded
-          if (!mbar_wait_bounded(p_full, jp & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN) ||
+          // P_{jp} written over S_{jp} (and O rescaled) by the softmax, V_{jp} loaded
+          if (!mbar_wait_bounded(&p_full[jp & 1], (jp >> 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN) ||
               !mbar_wait_bounded(v_full, jp & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN)) {
             *abort_flag = 1; ok = false; break;
           }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < BKV / 16; ++kk) {
-            mma_bf16_ss(t_o, smem_desc_sw128(pa + kk * 32, 16, 1024),
-                        smem_desc_sw128(va + kk * 16 * 128, KV_HALF, 1024), IDESC_PV, (jp > 0 || kk > 0) ? 1u : 0u);
+            const uint32_t a_tmem = tmem_base + static_cast<uint32_t>((jp & 1) * BKV + kk * 8);
+            mma_f16_ts(t_o, a_tmem, smem_desc_sw128(va + kk * 16 * 128, KV_HALF, 1024), IDESC_PV,
+                       (jp > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(pv_done);
           mma_commit(v_empty);
@@ -246,8 +264,6 @@ __global__ void __launch_bounds__(THREADS, 2) tp_attention_kernel(const __grid_c
     float m_ref = -INFINITY;   // reference max of the scaled scores (log2 units)
     float l_run = 0.f;
     bool ok = true;
-    uint8_t* p_row = sP + r * 128;
-    const int rsw = r & 7;
     for (int j = 0; j < nkv && ok; ++j) {
       const int ks = j & 1;
       // waits are made warp-uniform: tcgen05.ld/st are warp-collective instructions
@@ -287,14 +303,16 @@ __global__ void __launch_bounds__(THREADS, 2) tp_attention_kernel(const __grid_c
       }
       const bool move = mx > m_ref + RESCALE_LOG2;
       const float m_new = move ? mx : m_ref;
-      // P_{j-1} V_{j-1} must be done before P_j overwrites the P buffer and before O is rescaled
-      if (j > 0) {
+      // O is rescaled only after P_{j-1} V_{j-1} is done (P_j goes over S_j, so nothing
+      // else has to wait for it).  P_{j-2} V_{j-2} completed before S_j did, so the
+      // barrier is at most one phase behind and the parity wait is exact.
+      if (j > 0 && __any_sync(0xffffffffu, move)) {
         if (!__all_sync(0xffffffffu, mbar_wait_bounded(pv_done, (j - 1) & 1, a.wait_limit_ns, a.status,
                                                        WAIT_SITE_ATTN))) {
           *abort_flag = 1; ok = false; break;
         }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, move)) {
+        {
           const float alpha = move ? exp2f(m_ref - m_new) : 1.0f;
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
@@ -311,39 +329,35 @@ __global__ void __launch_bounds__(THREADS, 2) tp_attention_kernel(const __grid_c
       }
       const float m_use = m_new == -INFINITY ? 0.f : m_new;
       m_ref = m_new;
-      // P = exp2(s * scale - m) in fp16, written in the 128B-swizzled K-major layout (one
-      // 128-byte row per query); masked scores are -inf and give 0.  The row sum is taken
-      // over the fp32 values.
+      // P = exp2(s * scale - m) in fp16, two keys per 32-bit column, stored over the first
+      // 32 columns of S_j's buffer; masked scores are -inf and give 0.  The row sum is
+      // taken over the fp32 values.
       float ls0 = 0.f, ls1 = 0.f;
       const float neg_m = -m_use;
+      uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           float x0, x1;
           fma2_bc(x0, x1, __uint_as_float(sr[c][2 * i]), __uint_as_float(sr[c][2 * i + 1]), sl2, neg_m);
           const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
           add2_acc(ls0, ls1, e0, e1);
-          pk[i] = pack_f16x2(e0, e1);
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int chunk = c * 4 + u;   // 8 keys per 16-byte chunk
-          *reinterpret_cast<uint4*>(p_row + ((chunk ^ rsw) << 4)) =
-              make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+          pk[c * 16 + i] = pack_f16x2(e0, e1);
         }
       }
+      tmem_st_32x32b_x32(t_s, pk);
+      tmem_st_wait();
       const float lsum = ls0 + ls1;
       l_run += lsum;
-      // publish P_j to the tensor core (async proxy); S_j and O are released with it
-      fence_proxy_async_smem();
+      // publish P_j (tensor memory) to the tensor core; O is released with it
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[ks]);
     }
     if (ok && nkv > 0) {
-      if (__all_sync(0xffffffffu, mbar_wait_bounded(pv_done, (nkv - 1) & 1, a.wait_limit_ns, a.status,
-                                                    WAIT_SITE_ATTN))) {
+      // all of O is complete when the MMA thread's final commit (after the last P V) lands;
+      // pv_done could be two phases behind here, where its parity test is ambiguous
+      if (__all_sync(0xffffffffu, mbar_wait_bounded(drain_bar, 0, a.wait_limit_ns, a.status, WAIT_SITE_ATTN))) {
         tc_fence_after();
         const float inv = 1.f / l_run;
         uint16_t* dst = static_cast<uint16_t*>(a.O) + (static_cast<int64_t>(b) * a.S + q) * (a.H * D) + head * D;
