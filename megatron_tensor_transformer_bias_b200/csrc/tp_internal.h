@@ -104,6 +104,8 @@ tp_status launch_act(const float* x, float* y, int64_t n, int act, cudaStream_t 
 
 // Launch `kern` on `stream` with programmatic dependent launch (the kernel waits for
 // its predecessor with griddepcontrol.wait before touching global memory) and an
+// Record `msg` as the calling thread's tp_last_error() and return `s`.
+tp_status set_error(tp_status s, const char* msg);
 // optional cluster size.  TPB_PDL=0 turns the attribute off.
 bool pdl_enabled();
 template <typename... KArgs, typename... Args>
@@ -130,12 +132,12 @@ tp_status launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, 
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = n;
-  if (cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...) != cudaSuccess) return TP_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(TP_ERR_CUDA, cudaGetErrorString(e));
+  return TP_OK;
 }
 
-// Record `msg` as the calling thread's tp_last_error() and return `s`.
-tp_status set_error(tp_status s, const char* msg);
 
 // Launch tracing (tp_trace_*): brackets each kernel launch with events.
 void trace_before(cudaStream_t stream);
