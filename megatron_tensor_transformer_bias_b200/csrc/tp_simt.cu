@@ -62,6 +62,17 @@ __global__ void __launch_bounds__(256) reduce_partials_kernel(const float* __res
 // ---------------------------------------------------------------- layernorm
 constexpr int LN_THREADS = 256;
 
+// 8 consecutive bf16 values (16-byte aligned) as floats
+__device__ __forceinline__ void load_bf16x8(const uint16_t* p, float (&f)[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    f[2 * j] = __uint_as_float(w[j] << 16);
+    f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+  }
+}
+
 __device__ __forceinline__ float block_sum(float v, float* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -238,8 +249,120 @@ tp_status launch_reduce_partials(const float* P, int t, int64_t M, int64_t h, co
   return TP_OK;
 }
 
+// Register-resident LayerNorm for h <= 2048 * NCH: one 256-thread CTA per row, thread i
+// holds the 8-element chunks i, i + 256, ... (NCH of them) in registers.  Every load of
+// the row is issued before the first reduction, the mean and the variance are taken in
+// two exact passes over the registers, and gamma / beta are read 8 at a time.
+template <bool IN_F32, bool OUT_F16, int NCH>
+__global__ void __launch_bounds__(LN_THREADS) layernorm_reg_kernel(const void* __restrict__ x,
+                                                                   const uint16_t* __restrict__ g,
+                                                                   const uint16_t* __restrict__ b, int64_t h,
+                                                                   float eps, uint16_t* __restrict__ y) {
+  __shared__ float red[LN_THREADS / 32];
+  const int64_t r = blockIdx.x;
+  const int n8 = static_cast<int>(h / 8);
+  float f[NCH][8];
+  pdl_wait();
+#pragma unroll
+  for (int k = 0; k < NCH; ++k) {
+    const int v = threadIdx.x + k * LN_THREADS;
+    if (v < n8) {
+      if (IN_F32) {
+        const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(x) + r * h) + 2 * v;
+        const float4 a = __ldcs(p), c = __ldcs(p + 1);
+        f[k][0] = a.x; f[k][1] = a.y; f[k][2] = a.z; f[k][3] = a.w;
+        f[k][4] = c.x; f[k][5] = c.y; f[k][6] = c.z; f[k][7] = c.w;
+      } else {
+        const uint4 u = __ldcs(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + r * h) + v);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          f[k][2 * j] = __uint_as_float(w[j] << 16);
+          f[k][2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) f[k][j] = 0.f;
+    }
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int k = 0; k < NCH; ++k)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) s += f[k][j];
+  const float mean = block_sum(s, red) / static_cast<float>(h);
+  float q = 0.f;
+#pragma unroll
+  for (int k = 0; k < NCH; ++k) {
+    if (threadIdx.x + k * LN_THREADS < n8) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float d = f[k][j] - mean;
+        q += d * d;
+      }
+    }
+  }
+  const float var = block_sum(q, red) / static_cast<float>(h);
+  const float rstd = rsqrtf(var + eps);
+#pragma unroll
+  for (int k = 0; k < NCH; ++k) {
+    const int v = threadIdx.x + k * LN_THREADS;
+    if (v >= n8) continue;
+    float gg[8], bb[8];
+    if (g) {
+      load_bf16x8(g + 8 * static_cast<int64_t>(v), gg);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) gg[j] = 1.f;
+    }
+    if (b) {
+      load_bf16x8(b + 8 * static_cast<int64_t>(v), bb);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) bb[j] = 0.f;
+    }
+    float o[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) o[j] = (f[k][j] - mean) * rstd * gg[j] + bb[j];
+    uint4 u;
+    if (OUT_F16) {
+      u.x = pack_f16x2(o[0], o[1]); u.y = pack_f16x2(o[2], o[3]);
+      u.z = pack_f16x2(o[4], o[5]); u.w = pack_f16x2(o[6], o[7]);
+    } else {
+      u.x = pack_bf16x2(o[0], o[1]); u.y = pack_bf16x2(o[2], o[3]);
+      u.z = pack_bf16x2(o[4], o[5]); u.w = pack_bf16x2(o[6], o[7]);
+    }
+    reinterpret_cast<uint4*>(y + r * h)[v] = u;
+  }
+  pdl_launch_dependents();
+}
+
+template <int NCH>
+static tp_status launch_layernorm_reg(const void* x, int in_fp32, const void* g, const void* b, int64_t M, int64_t h,
+                                      float eps, void* y, int out_f16, cudaStream_t stream) {
+  const int key = (in_fp32 ? 1 : 0) | (out_f16 ? 2 : 0);
+  void (*kern)(const void*, const uint16_t*, const uint16_t*, int64_t, float, uint16_t*) =
+      key == 0   ? layernorm_reg_kernel<false, false, NCH>
+      : key == 1 ? layernorm_reg_kernel<true, false, NCH>
+      : key == 2 ? layernorm_reg_kernel<false, true, NCH>
+                 : layernorm_reg_kernel<true, true, NCH>;
+  trace_before(stream);
+  const tp_status st = launch_ex(kern, dim3(static_cast<unsigned>(M)), dim3(LN_THREADS), 0, stream, 1, x,
+                                 static_cast<const uint16_t*>(g), static_cast<const uint16_t*>(b), h, eps,
+                                 static_cast<uint16_t*>(y));
+  if (st != TP_OK) return st;
+  trace_after(stream, "layernorm");
+  return TP_OK;
+}
+
 tp_status launch_layernorm(const void* x, int in_fp32, const void* g, const void* b, int64_t M, int64_t h,
                            float eps, void* y, int out_f16, cudaStream_t stream) {
+  if (M > 0 && h <= 8 * LN_THREADS * 4) {
+    if (h <= 8 * LN_THREADS) return launch_layernorm_reg<1>(x, in_fp32, g, b, M, h, eps, y, out_f16, stream);
+    if (h <= 8 * LN_THREADS * 2) return launch_layernorm_reg<2>(x, in_fp32, g, b, M, h, eps, y, out_f16, stream);
+    return launch_layernorm_reg<4>(x, in_fp32, g, b, M, h, eps, y, out_f16, stream);
+  }
   if (M == 0) return TP_OK;
   const size_t smem = static_cast<size_t>(h) * sizeof(float);
   const int key = (in_fp32 ? 1 : 0) | (out_f16 ? 2 : 0);
