@@ -12,7 +12,10 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-@pytest.mark.parametrize("M,h", [(1, 8), (37, 256), (2048, 8192), (5, 22528)])
+# h <= 2048, <= 4096 and <= 8192 take the register-resident kernel with 1, 2 and 4 chunks of
+# 8 per thread (5000: some threads hold a third chunk, none a fourth); above 8192 the row is
+# cached in shared memory.
+@pytest.mark.parametrize("M,h", [(1, 8), (37, 256), (3, 4000), (7, 5000), (2048, 8192), (2, 8200), (5, 22528)])
 @pytest.mark.parametrize("in_dtype", [torch.bfloat16, torch.float32])
 def test_layernorm(M, h, in_dtype):
     g = torch.Generator(device=DEV).manual_seed(M * 7 + h)
