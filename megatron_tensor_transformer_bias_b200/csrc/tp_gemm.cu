@@ -540,13 +540,19 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
         const TileCoord tc = tile_coord(a, tile, m_tiles, n_tiles);
         const int m0 = tc.m_blk * P_ROWS + static_cast<int>(rank) * BM;
         const int n0 = tc.n_blk * BN + static_cast<int>(rank) * (BN / 2);
+        // Row layer: the K loop runs backwards in even rounds of tiles and forwards in odd
+        // ones, so each round starts on the K-slices of A that are still in L2 -- the end
+        // of K for the first round (the producing layer wrote it last), the start for the
+        // second (the first round read it last), and so on.  The order is fixed per tile.
+        const bool rev = a.concat && (((tile - cid) / nclusters) & 1) == 0;
         for (int it = 0; it < k_iters; ++it) {
           if (*abort_flag) { ok = false; break; }
           if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, a.wait_limit_ns, a.status, WAIT_SITE_PRODUCER)) {
             *abort_flag = 1; ok = false; break;
           }
-          const int g = a.concat ? it / kb_per_group : tc.g;
-          const int kb = a.concat ? it - g * kb_per_group : it;
+          const int kidx = rev ? k_iters - 1 - it : it;
+          const int g = a.concat ? kidx / kb_per_group : tc.g;
+          const int kb = a.concat ? kidx - g * kb_per_group : kidx;
           const uint32_t fb = full0_leader + static_cast<uint32_t>(stage) * 8u;
           if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * P_STAGE_BYTES);
           tma_load_2d_pair(sA + stage * P_A_BYTES, &a.tmA, fb, g * a.a_k_per_group + kb * BK, m0, pol_a);
