@@ -7,16 +7,20 @@
 // epilogue adds the shard's bias and applies the element-wise nonlinearity
 // straight from TMEM (no communication is needed, the nonlinearity is local).
 // Row-parallel layer (steps 2-3): either one tile per (m-block, n-block) whose
-// K loop walks the K-slices of shards 0..t-1 in order into the same TMEM
-// accumulator (the reduction happens in the accumulator) with a bias + residual
-// epilogue, or one tile per (shard, m, n) writing fp32 partials.
+// K loop walks the K-slices of all shards into the same TMEM accumulator (the
+// reduction happens in the accumulator) with a bias + residual epilogue, or one
+// tile per (shard, m, n) writing fp32 partials.
 //
-// Roles per CTA (192 threads, one CTA per SM):
-//   warp 0      TMA producer: A tile 128x64 and B tile 64x256 per stage
-//   warp 1      TMEM allocation; one thread issues tcgen05.mma (M=128, N=256, K=16)
-//   warps 2..5  epilogue: tcgen05.ld TMEM -> registers -> bias/act/residual -> global
-// A 4-stage shared-memory ring feeds the MMA; two 256-column TMEM accumulators let
-// the epilogue of one tile overlap the main loop of the next.
+// Two kernels share the roles below: tp_gemm_pair_kernel (the default; a cluster
+// of two CTAs computes a 256x256 tile with cta_group::2 MMAs) and tp_gemm_kernel
+// (one CTA, 128x256 tiles).  Roles per CTA (320 threads, one CTA per SM):
+//   warp 0      TMA producer: this CTA's operand tiles, one 64-wide K step per stage
+//   warp 1      TMEM allocation; one thread issues tcgen05.mma (16-deep K per instruction)
+//   warps 2..9  epilogue: tcgen05.ld TMEM -> registers -> bias/act/residual -> global
+//               (16-bit outputs through swizzled shared-memory staging and TMA stores)
+// A shared-memory ring (6 stages for pairs, 4 for one CTA) feeds the MMA; two
+// 256-column TMEM accumulators let the epilogue of one tile overlap the main loop
+// of the next.
 #include <cstdlib>
 
 #include "tp_internal.h"
