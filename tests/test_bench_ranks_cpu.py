@@ -58,3 +58,14 @@ def test_reference_arm_runs_on_cpu(capsys, monkeypatch):
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_kernel_source_hash_ignores_comments_only():
+    """The ncu figures are keyed on the kernel sources without comments and layout: a
+    comment edit keeps them, any code edit drops them."""
+    import bench
+    code = "int f(int a) {\n  return a + 1;  // one more\n}\n/* block\n   comment */\n"
+    assert bench._code_only(code) == "int f(int a) { return a + 1; }"
+    assert bench._code_only(code.replace("// one more", "// a different note")) == bench._code_only(code)
+    assert bench._code_only(code.replace("a + 1", "a + 2")) != bench._code_only(code)
+    assert len(bench._csrc_sha()) == 16
