@@ -15,7 +15,7 @@
  *   adds between the sub-layers.
  *
  * All t logical shards run on the one GPU; step 3 becomes an on-device
- * reduction (fixed order i = 0..t-1, no atomics, bitwise reproducible).
+ * reduction in a fixed order (no atomics, bitwise reproducible).
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -69,8 +69,11 @@ typedef enum { TP_BF16 = 0, TP_FP32 = 1, TP_FP16 = 2 } tp_dtype;
 
 /* How step 3 (the all-reduce) is done on one device.
  * TP_REDUCE_FUSED:    one row-GEMM tile accumulates the K-slices of all t
- *                     shards in order into one fp32 accumulator, and its
- *                     epilogue adds the bias and the residual.
+ *                     shards into one fp32 accumulator, in a fixed order that
+ *                     depends only on the tile's place in the schedule
+ *                     (ascending or descending K, whichever starts on data
+ *                     still in L2), and its epilogue adds the bias and the
+ *                     residual.  The result is the same bits for every t.
  * TP_REDUCE_PARTIALS: the row GEMM writes t fp32 partials Y_i [t, M, h] to the
  *                     workspace; a reduce kernel sums them in order 0..t-1
  *                     and adds bias and residual. */
