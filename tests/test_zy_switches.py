@@ -1,0 +1,31 @@
+"""The library's launch switches, read once per process from the environment:
+TPB_GEMM_PAIRS=0 runs every GEMM on the one-CTA kernel (128x256 tiles) instead of CTA
+pairs, TPB_PDL=0 launches without programmatic dependent launch.  Each is exercised by
+re-running small parity tests against the oracle in a child process."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+# small, every-element parity cases of the FFN (both reduce modes, fp16 W2, ragged M),
+# the linears, attention (causal and not) and the layer
+CASES = [
+    "tests/test_gpu_ffn.py::test_bf16_small_full",
+    "tests/test_gpu_ffn.py::test_bf16_sharding_invariance_bitwise_and_determinism",
+    "tests/test_gpu_ffn.py::test_column_linear",
+    "tests/test_gpu_ffn.py::test_row_linear",
+    "tests/test_gpu_attention_layer.py::test_attention_small_full",
+    "tests/test_gpu_attention_layer.py::test_layer_small_full",
+]
+
+
+@pytest.mark.parametrize("env", [{"TPB_GEMM_PAIRS": "0"}, {"TPB_PDL": "0"}], ids=["one_cta_gemm", "no_pdl"])
+def test_parity_under_switch(env):
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider", *CASES],
+                       cwd=ROOT, env=dict(os.environ, **env), capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
