@@ -183,3 +183,32 @@ def test_ffn_hidden_sweep_sampled(h):
         assert_bf16_close(out[rows], ref, f"M4096 h{h} t{t}")
     del inp, out
     torch.cuda.empty_cache()
+
+
+def test_column_gelu_closed_forms_identity_weights():
+    """With W1 = I and no bias the column layer's epilogue output is GeLU(X) element by
+    element (fp16 operands and output): GeLU(0) = 0, table values of z * Phi(z),
+    GeLU(z) - GeLU(-z) = z, GeLU(z) = z and GeLU(-z) = 0 far in the tails."""
+    h, t = 256, 2
+    g = torch.Generator(device=DEV).manual_seed(23)
+    z = torch.randn(64, h // 2, generator=g, device=DEV) * 3
+    table = torch.tensor([0.0, 1.0, 2.0, 0.5, 16.0], device=DEV)
+    z[0, :5] = table
+    X = torch.cat([z, -z], dim=1).to(torch.float16)       # columns j and j + h/2 hold z and -z
+    W = torch.eye(h, device=DEV).to(torch.float16)
+    out = torch.empty(64, h, dtype=torch.float16, device=DEV)
+    tb.tp_column_linear_forward(X, tb.shard_columns(W, t), None, out, act="gelu")
+    got = to64(out)
+    x = to64(X)
+    assert got[0, 0] == 0.0 and got[0, h // 2] == 0.0
+    ulp = 2.0 ** -10
+    for col, phi in [(1, 0.8413447460685429), (2, 0.9772498680518208), (3, 0.6914624612740131)]:
+        want = x[0, col] * phi
+        assert abs(got[0, col] - want) <= ulp * abs(want), (col, got[0, col], want)
+    assert got[0, 4] == 16.0 and got[0, 4 + h // 2] == 0.0
+    half = h // 2
+    # odd part: GeLU(z) - GeLU(-z) = z, each side rounded once to fp16
+    d = got[:, :half] - got[:, half:]
+    assert np.all(np.abs(d - x[:, :half]) <= ulp * (np.abs(got[:, :half]) + np.abs(got[:, half:])) + 1e-7)
+    ref = oracle.gelu(x)
+    assert np.all(np.abs(got - ref) <= ulp * np.abs(ref) + 1e-7)
