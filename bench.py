@@ -65,15 +65,44 @@ def _csrc_sha():
     return h.hexdigest()[:16]
 
 
+# The sources that define each traced launch: its kernel file, the shared device helpers
+# and declarations, and the host code that builds its launch (tensor maps, grid, workspace).
+_SHARED_SOURCES = ["tp_ptx.cuh", "tp_internal.h", "tp_api.cu"]
+KERNEL_SOURCES = {
+    "gemm_column_act": ["tp_gemm.cu"] + _SHARED_SOURCES,
+    "gemm_row_fused_reduce": ["tp_gemm.cu"] + _SHARED_SOURCES,
+    "gemm_row_partials": ["tp_gemm.cu"] + _SHARED_SOURCES,
+    "gemm_qkv": ["tp_gemm.cu"] + _SHARED_SOURCES,
+    "attention": ["tp_attention.cu"] + _SHARED_SOURCES,
+    "reduce_partials": ["tp_simt.cu"] + _SHARED_SOURCES,
+    "layernorm": ["tp_simt.cu"] + _SHARED_SOURCES,
+}
+
+
+def _kernel_sha(kernel):
+    """Hash of the sources (comments and layout ignored) that define one traced launch;
+    the whole source tree for a launch not listed."""
+    files = KERNEL_SOURCES.get(kernel)
+    if not files:
+        return _csrc_sha()
+    d = os.path.join(ROOT, "megatron_tensor_transformer_bias_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(files):
+        with open(os.path.join(d, f), encoding="utf-8") as fh:
+            h.update(f.encode() + _code_only(fh.read()).encode())
+    return h.hexdigest()[:16]
+
+
 def _traffic(workload, kernel):
-    """DRAM bytes per launch from the committed ncu capture, or None if the kernels changed since."""
+    """DRAM bytes per launch from the committed ncu capture, or None if the sources that
+    define the kernel changed since."""
     try:
         with open(os.path.join(PROFILES, "ncu_traffic.json")) as fh:
             t = json.load(fh)
     except Exception:
         return None
     rec = t.get(f"{workload}:{kernel}")
-    if not rec or rec.get("csrc_sha") != _csrc_sha():
+    if not rec or rec.get("src_sha") != _kernel_sha(kernel):
         return None
     return rec["dram_bytes_per_launch"]
 

@@ -69,3 +69,7 @@ def test_kernel_source_hash_ignores_comments_only():
     assert bench._code_only(code.replace("// one more", "// a different note")) == bench._code_only(code)
     assert bench._code_only(code.replace("a + 1", "a + 2")) != bench._code_only(code)
     assert len(bench._csrc_sha()) == 16
+    # each launch is keyed on the sources that define it
+    assert bench._kernel_sha("attention") != bench._kernel_sha("gemm_row_fused_reduce")
+    assert bench._kernel_sha("gemm_column_act") == bench._kernel_sha("gemm_row_fused_reduce")
+    assert bench._kernel_sha("not_a_kernel") == bench._csrc_sha()
