@@ -12,6 +12,11 @@ their bf16 (or fp32) bits, with no intermediate rounding.  Matrix products use
 numpy's matmul and erf comes from ``scipy.special``; no blocking, fusion or
 reordering is added beyond what the definitions state.
 
+The backward pass of the FFN block (gradients of the forward block by the
+chain rule, with the sum over shards of the column layer's input gradient as
+its one reduction) is pinned the same way: a normal-table check of GeLU',
+central finite differences, float64 autograd and sharding invariance.
+
 Source of the method: the page "Tensor Parallelism > Combining Column and Row
 Parallelism" (mbrenndoerfer.com), cited below as [TP-CR] with its numbered
 steps (1 column-parallel W1, 2 row-parallel W2, 3 all-reduce) and its
@@ -34,4 +39,8 @@ from .tp_block import (  # noqa: F401
     attn_forward_sharded,
     layer_forward,
     reduce_partials,
+    gelu_grad,
+    relu_grad,
+    ffn_backward,
+    ffn_backward_sharded,
 )

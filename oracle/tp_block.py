@@ -252,3 +252,77 @@ def layer_forward(X, p, B, S, H, d, eps=1e-5, causal=True, rows=None):
     h1 = X[rows] + attn_rows
     a2 = layernorm(h1, p["ln2_g"], p["ln2_b"], eps)
     return ffn_forward(a2, p["W1"], p["b1"], p["W2"], p["b2"], h1)
+
+
+# --------------------------------------------------------------------------
+# Backward pass of the FFN block.  The page describes the forward pass (one
+# all-reduce per two-layer block) and notes its effect on training; the
+# gradients are the chain rule taken back through steps 3, 2 and 1.  Read with
+# the chaining paragraph's column/row duality: the upstream gradient dY is the
+# same on every shard (it is the gradient of the forward all-reduce's output),
+# so the row-parallel layer's input gradient dA_i = dY W2_i^T is local to shard
+# i, while the column-parallel layer's input gradient dX = sum_i dZ_i W1_i^T is
+# a sum over shards -- the backward pass's one reduction.
+# --------------------------------------------------------------------------
+def gelu_grad(z):
+    """d/dz GeLU(z) = Phi(z) + z phi(z), phi(z) = exp(-z^2/2) / sqrt(2 pi) the normal density."""
+    z = _f64(z)
+    return 0.5 * (1.0 + _erf(z / math.sqrt(2.0))) + z * np.exp(-0.5 * z * z) / math.sqrt(2.0 * math.pi)
+
+
+def relu_grad(z):
+    """d/dz ReLU(z): 1 where z > 0, else 0 (0 at z = 0)."""
+    return (_f64(z) > 0.0).astype(F64)
+
+
+_ACT_GRAD = {"gelu": gelu_grad, "relu": relu_grad}
+
+
+def ffn_backward(X, W1, b1, W2, dY, act="gelu"):
+    """Gradients of out = act(X W1 + b1) W2 + b2 + R given dY = dL/d(out).
+
+    Returns a dict with dX (the gradient through the FFN path only: when the
+    residual R is X, the caller's total input gradient is dX + dY), dW1, db1,
+    dW2 and db2:
+        Z = X W1 + b1,   A = act(Z)
+        dW2 = A^T dY,    db2 = sum over rows of dY
+        dA = dY W2^T,    dZ = dA * act'(Z)
+        dW1 = X^T dZ,    db1 = sum over rows of dZ,   dX = dZ W1^T
+    """
+    X, W1, W2, dY = _f64(X), _f64(W1), _f64(W2), _f64(dY)
+    Z = X @ W1
+    if b1 is not None:
+        Z = Z + _f64(b1)
+    A = _ACT[act](Z)
+    dA = dY @ W2.T
+    dZ = dA * _ACT_GRAD[act](Z)
+    return {"dX": dZ @ W1.T, "dW1": X.T @ dZ, "db1": dZ.sum(axis=0), "dW2": A.T @ dY, "db2": dY.sum(axis=0)}
+
+
+def ffn_backward_sharded(X, shards: Iterable[Tuple], dY, act="gelu"):
+    """The backward pass shard by shard, for ``shards`` yielding (W1_i, b1_i or None, W2_i)
+    in the order 0..t-1:
+
+    * recompute Z_i = X W1_i (+ b1_i) and A_i = act(Z_i) (step 1 again, local);
+    * dW2_i = A_i^T dY and dA_i = dY W2_i^T (the row layer's gradients, local);
+    * dZ_i = dA_i * act'(Z_i), dW1_i = X^T dZ_i, db1_i = column sums of dZ_i (local);
+    * dX = sum_i dZ_i W1_i^T, taken in the order 0..t-1 (the reduction);
+    * db2 = column sums of dY, once.
+
+    Returns (dX, [dW1_i], [db1_i], [dW2_i], db2)."""
+    X, dY = _f64(X), _f64(dY)
+    dX = None
+    dW1, db1, dW2 = [], [], []
+    for W1_i, b1_i, W2_i in shards:
+        W1_i, W2_i = _f64(W1_i), _f64(W2_i)
+        Z_i = X @ W1_i
+        if b1_i is not None:
+            Z_i = Z_i + _f64(b1_i)
+        A_i = _ACT[act](Z_i)
+        dW2.append(A_i.T @ dY)
+        dZ_i = (dY @ W2_i.T) * _ACT_GRAD[act](Z_i)
+        dW1.append(X.T @ dZ_i)
+        db1.append(dZ_i.sum(axis=0))
+        part = dZ_i @ W1_i.T
+        dX = part if dX is None else dX + part
+    return dX, dW1, db1, dW2, dY.sum(axis=0)

@@ -98,3 +98,37 @@ def test_missing_layernorm_in_layer_is_caught(monkeypatch):
         return np.asarray(x, float)
     monkeypatch.setattr(tb, "layernorm", identity_ln)
     _expect_fail(pins.check_layer)
+
+
+def test_gelu_grad_without_density_term_is_caught(monkeypatch):
+    # Phi(z) alone, the derivative with the z phi(z) term dropped
+    monkeypatch.setattr(tb, "gelu_grad", lambda z: 0.5 * (1.0 + tb._erf(np.asarray(z, float) / math.sqrt(2.0))))
+    monkeypatch.setattr(oracle, "gelu_grad", tb.gelu_grad)
+    monkeypatch.setitem(tb._ACT_GRAD, "gelu", tb.gelu_grad)
+    _expect_fail(pins.check_gelu_grad)
+    _expect_fail(pins.check_ffn_backward_finite_differences)
+
+
+def test_dw2_from_preactivation_is_caught(monkeypatch):
+    real = tb.ffn_backward
+
+    def dw2_from_z(X, W1, b1, W2, dY, act="gelu"):
+        g = real(X, W1, b1, W2, dY, act)
+        Z = np.asarray(X, float) @ np.asarray(W1, float) + np.asarray(b1, float)
+        g["dW2"] = Z.T @ np.asarray(dY, float)
+        return g
+    monkeypatch.setattr(oracle, "ffn_backward", dw2_from_z)
+    _expect_fail(pins.check_ffn_backward_finite_differences)
+
+
+def test_input_gradient_missing_a_shard_is_caught(monkeypatch):
+    real = tb.ffn_backward_sharded
+
+    def drop_last_shard_from_dx(X, shards, dY, act="gelu"):
+        shards = list(shards)
+        dX, dW1, db1, dW2, db2 = real(X, shards, dY, act)
+        W1_l, b1_l, W2_l = shards[-1]
+        dX_l, *_ = real(X, [shards[-1]], dY, act)
+        return dX - dX_l if len(shards) > 1 else dX, dW1, db1, dW2, db2
+    monkeypatch.setattr(oracle, "ffn_backward_sharded", drop_last_shard_from_dx)
+    _expect_fail(pins.check_ffn_backward_sharding)

@@ -393,3 +393,113 @@ def test_sample_rows():
     assert {0, 2047, 2048, 4095} <= set(rows)
     assert rows == inputs.sample_rows(4096, 64, seq=2048)
     assert inputs.sample_rows(5, 64) == [0, 1, 2, 3, 4]
+
+
+# ---------------------------------------------------------------- FFN backward
+def _normal_density(x):
+    return math.exp(-0.5 * x * x) / math.sqrt(2.0 * math.pi)
+
+
+def check_gelu_grad():
+    """GeLU'(x) = Phi(x) + x phi(x): Phi from the printed normal table (not from erf),
+    phi the normal density; GeLU'(0) = 1/2; GeLU'(x) + GeLU'(-x) = 1 (derivative of
+    GeLU(x) - GeLU(-x) = x); -> 1 and -> 0 in the tails; and the derivative of the
+    oracle's own GeLU by central differences."""
+    for x, phi in _phi_table():
+        want = phi + x * _normal_density(x)
+        assert abs(oracle.gelu_grad(x) - want) <= 1e-14, (x, oracle.gelu_grad(x), want)
+        want_neg = (1.0 - phi) - x * _normal_density(x)
+        assert abs(oracle.gelu_grad(-x) - want_neg) <= 1e-14, x
+    assert oracle.gelu_grad(0.0) == 0.5
+    x = np.linspace(-7, 7, 1401)
+    np.testing.assert_allclose(oracle.gelu_grad(x) + oracle.gelu_grad(-x), 1.0, rtol=0, atol=1e-14)
+    assert abs(oracle.gelu_grad(12.0) - 1.0) < 1e-15 and abs(oracle.gelu_grad(-12.0)) < 1e-15
+    h = 1e-5
+    fd = (oracle.gelu(x + h) - oracle.gelu(x - h)) / (2 * h)
+    np.testing.assert_allclose(oracle.gelu_grad(x), fd, rtol=0, atol=1e-9)
+
+
+def test_gelu_grad():
+    check_gelu_grad()
+
+
+def test_relu_grad():
+    np.testing.assert_array_equal(oracle.relu_grad(np.array([-1.0, 0.0, 1e-30, 2.0])), [0.0, 0.0, 1.0, 1.0])
+
+
+def _tiny_backward_case(seed=21, M=3, h=4, f=6):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((M, h)), rng.standard_normal((h, f)) * 0.5, rng.standard_normal(f) * 0.3,
+            rng.standard_normal((f, h)) * 0.5, rng.standard_normal(h) * 0.3, rng.standard_normal((M, h)))
+
+
+def check_ffn_backward_finite_differences(act="gelu"):
+    """Every gradient entry of L = sum(dY * out) against a central difference of the
+    oracle's own forward, on a tiny block (no shared code with the backward)."""
+    X, W1, b1, W2, b2, dY = _tiny_backward_case()
+    g = oracle.ffn_backward(X, W1, b1, W2, dY, act=act)
+
+    def loss(X_, W1_, b1_, W2_, b2_):
+        return float(np.sum(dY * oracle.ffn_forward(X_, W1_, b1_, W2_, b2_, None, act=act)))
+
+    args = [X, W1, b1, W2, b2]
+    names = ["dX", "dW1", "db1", "dW2", "db2"]
+    eps = 1e-6
+    for k, name in enumerate(names):
+        a = args[k]
+        fd = np.zeros_like(a)
+        for idx in np.ndindex(a.shape):
+            up = [x.copy() for x in args]
+            dn = [x.copy() for x in args]
+            up[k][idx] += eps
+            dn[k][idx] -= eps
+            fd[idx] = (loss(*up) - loss(*dn)) / (2 * eps)
+        np.testing.assert_allclose(g[name], fd, rtol=1e-6, atol=1e-7, err_msg=name)
+
+
+def test_ffn_backward_finite_differences():
+    check_ffn_backward_finite_differences("gelu")
+    check_ffn_backward_finite_differences("relu")
+
+
+def test_ffn_backward_matches_float64_autograd():
+    X, W1, b1, W2, b2, dY = _tiny_backward_case(seed=22, M=5, h=8, f=12)
+    t = [torch.tensor(a, dtype=torch.float64, requires_grad=True) for a in (X, W1, b1, W2, b2)]
+    out = F.gelu(t[0] @ t[1] + t[2], approximate="none") @ t[3] + t[4]
+    out.backward(torch.tensor(dY))
+    g = oracle.ffn_backward(X, W1, b1, W2, dY)
+    for name, tt in zip(["dX", "dW1", "db1", "dW2", "db2"], t):
+        np.testing.assert_allclose(g[name], tt.grad.numpy(), rtol=1e-12, atol=1e-13, err_msg=name)
+
+
+def check_ffn_backward_sharding():
+    """The shard-by-shard backward (local row-layer gradients, one ordered sum for the
+    input gradient) equals the unsharded chain rule for every t dividing f."""
+    X, W1, b1, W2, b2, dY = _tiny_backward_case(seed=23, M=7, h=8, f=24)
+    g = oracle.ffn_backward(X, W1, b1, W2, dY)
+    for t in (1, 2, 3, 4, 6, 8, 12, 24):
+        n = 24 // t
+        shards = [(W1[:, i * n:(i + 1) * n], b1[i * n:(i + 1) * n], W2[i * n:(i + 1) * n]) for i in range(t)]
+        dX, dW1, db1, dW2, db2 = oracle.ffn_backward_sharded(X, shards, dY)
+        np.testing.assert_allclose(dX, g["dX"], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(np.concatenate(dW1, axis=1), g["dW1"], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(np.concatenate(db1), g["db1"], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(np.concatenate(dW2, axis=0), g["dW2"], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(db2, g["db2"], rtol=0, atol=1e-12)
+
+
+def test_ffn_backward_sharding():
+    check_ffn_backward_sharding()
+
+
+def test_ffn_backward_special_cases():
+    X, W1, b1, W2, b2, dY = _tiny_backward_case(seed=24)
+    z = oracle.ffn_backward(X, W1, b1, W2, np.zeros_like(dY))
+    for v in z.values():
+        assert not np.any(v)
+    # W2 = 0: nothing flows back into the column layer; the row layer still gets A^T dY
+    g = oracle.ffn_backward(X, W1, b1, np.zeros_like(W2), dY)
+    assert not np.any(g["dX"]) and not np.any(g["dW1"]) and not np.any(g["db1"])
+    A = oracle.gelu(X @ W1 + b1)
+    np.testing.assert_allclose(g["dW2"], A.T @ dY, rtol=1e-14)
+    np.testing.assert_allclose(g["db2"], dY.sum(0), rtol=1e-14)
