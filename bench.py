@@ -1,22 +1,26 @@
 """Throughput of the column->row tensor-parallel block on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload ffn|attn|layer|sweep] [--t T] [--h H] [--mode fused|partials]
+                    [--workload all|ffn|bwd|attn|layer|sweep|fp32] [--t T] [--h H|all]
+                    [--mode fused|partials] [--no-cpu-baseline] [--no-sustained]
 
-Default step (the headline): one forward of the FFN block -- column-parallel
-GEMM + bias + exact GeLU, row-parallel GEMM, on-device reduction of the t
-logical shards + bias + residual -- at M=2048 tokens (batch 4 x seq 512),
-h=4096, f=16384, t=4, bf16 with fp32 accumulation, seeded synthetic inputs.
-Metric: TFLOP/s with the algorithmic count 4*M*h*f per step.  Other workloads
-(the attention sub-layer, the pre-LN layer, the FFN hidden-size sweep) print the
-same line for their own algorithmic FLOP count.
+Default (``--workload all``): one JSON line per workload, the headline last --
+the tiny fp32 FFN block, the attention sub-layer, the pre-LN layer, the FFN
+hidden-size sweep at h = 22528 for t = 1 and 8, the FFN block's backward pass,
+the FFN block with the partials reduction, and finally the headline: one
+forward of the FFN block --
+column-parallel GEMM + bias + exact GeLU, row-parallel GEMM, on-device reduction
+of the t logical shards + bias + residual -- at M=2048 tokens (batch 4 x seq
+512), h=4096, f=16384, t=4, bf16 with fp32 accumulation, seeded synthetic
+inputs.  Metric: TFLOP/s with the algorithmic count (the GEMMs, 2*M*K*N each,
+and causal attention 4*B*H*d*S(S+1)/2) per step.
 
 Under torchrun each rank runs an independent replica on its own GPU (its own
 token batch, no data-path collective); the value is the total work over all
 ranks divided by the slowest rank's device time.
 
 ``--impl reference`` times the fp64 CPU oracle instead (rank 0 only), on a
-bounded sample of token rows per step.
+bounded sample of token rows per step of the same workloads.
 """
 from __future__ import annotations
 
@@ -35,6 +39,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "TFLOP/s & % of BF16 peak, column→row TP FFN block (t=4 shards), 1 B200"
 PROFILES = os.path.join(ROOT, "profiles")
+DATA = "synthetic (seeded randn; X~N(0,1), W~N(0,0.02^2), b~N(0,0.01^2), residual=X)"
 
 
 def _peaks():
@@ -43,9 +48,11 @@ def _peaks():
         with open(path) as fh:
             p = json.load(fh)
         return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
-                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "source": "measured"}
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "sm_max_mhz": p.get("sm_max_mhz", 1965.0), "source": "measured"}
     except Exception:
-        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0,
+                "source": "fallback"}
 
 
 def _code_only(src: str) -> str:
@@ -174,45 +181,97 @@ class ClockSampler:
         return out
 
 
+# ---------------------------------------------------------------- host facts
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max(i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas")
+    except Exception:
+        return os.cpu_count()
+
+
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return None
+
+
+def _host():
+    return {"cores": _blas_threads(), "host_cpus": os.cpu_count(), "cpu_model": _cpu_model()}
+
+
+def _to64(t):
+    import torch
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
 # ---------------------------------------------------------------- workloads
 class Workload:
-    """One step of a workload: `step(X_dev, out_dev)` runs it through the C ABI."""
+    """One step of a workload: `step(X_dev, out_dev, stream)` runs it through the C ABI.
+
+    `oracle_setup(dev)` builds the host-side state of the oracle (fp64 copies of the
+    inputs, or chunk sources for the largest sizes); `oracle_rows(state, rng, n)` runs
+    the oracle as it stands on a sample of about n output rows and returns the
+    algorithmic FLOPs that sample stands for (rows / M of the workload's count)."""
     name = ""
     flops = 0
+    dtype = "bf16"
     kernel_amount = {}   # kernel name -> (bound, algorithmic amount per launch, unit)
+    ref_rows = 8         # token rows per step of the reference arm
 
     def config(self):
         return {"workload": self.name}
 
+    def metric(self):
+        return f"TFLOP/s, {self.name}, 1 B200"
+
 
 class FFN(Workload):
-    def __init__(self, w, mode, w2_fp16=False):
-        self.w, self.mode, self.w2_fp16 = w, mode, w2_fp16
-        self.name = w.name + ("" if mode == "fused" else "_partials") + ("_w2fp16" if w2_fp16 else "")
+    def __init__(self, w, mode, w2_fp16=False, headline=False):
+        self.w, self.mode, self.w2_fp16, self.headline = w, mode, w2_fp16, headline
+        # the fp32 block always sums fp32 partials; its name carries no mode
+        self.name = w.name + ("" if mode == "fused" or w.dtype == "fp32" else "_partials") + \
+            ("_w2fp16" if w2_fp16 else "")
         self.flops = w.flops
+        self.dtype = "bf16" if w.dtype == "bf16" else "f32"
+        if w.dtype == "bf16" and w2_fp16:
+            self.dtype = "bf16 (fp16 act(Z))"
         M, h, f, t = w.M, w.h, w.f, w.t
         self.kernel_amount = {
             "gemm_column_act": ("tensor", 2 * M * h * f, "FLOP"),
             "gemm_row_fused_reduce": ("tensor", 2 * M * f * h, "FLOP"),
             "gemm_row_partials": ("tensor", 2 * M * f * h, "FLOP"),
             "reduce_partials": ("hbm", (4 * t + 2 + 2) * M * h + 2 * h, "B"),
+            # fp32 workload: FFMA on the CUDA cores (2 FLOP per FMA)
+            "f32_col_gemm": ("alu", 2 * M * h * f, "FLOP"),
+            "f32_row_gemm": ("alu", 2 * M * f * h, "FLOP"),
         }
+
+    def metric(self):
+        return METRIC if self.headline else super().metric()
 
     def setup(self, dev, rank):
         import torch
         from megatron_tensor_transformer_bias_b200 import inputs
         from megatron_tensor_transformer_bias_b200 import tpblock as tb
         w = self.w
-        p = inputs.ffn_inputs(w.M, w.h, w.f, "bf16", seed=0, device=dev)
+        p = inputs.ffn_inputs(w.M, w.h, w.f, w.dtype, seed=0, device=dev)
         if rank:  # each replica runs its own token batch (same weights)
             g = torch.Generator(device=dev).manual_seed(7919 * rank)
-            p["X"] = torch.randn(w.M, w.h, generator=g, device=dev).to(torch.bfloat16)
+            p["X"] = torch.randn(w.M, w.h, generator=g, device=dev).to(p["X"].dtype)
+        self.p = p
         W2 = inputs.as_fp16(p["W2"]) if self.w2_fp16 else p["W2"]
         self.W1 = tb.shard_columns(p["W1"], w.t)
         self.W2 = tb.shard_rows(W2, w.t)
         self.b1 = tb.shard_vector(p["b1"], w.t)
         self.b2 = p["b2"]
-        self.ws = tb.workspace(tb.tp_ffn_workspace_bytes(w.M, w.h, w.f, w.t, tb.TP_BF16, tb.MODES[self.mode]), dev)
+        dt = tb.TP_FP32 if w.dtype == "fp32" else tb.TP_BF16
+        self.ws = tb.workspace(tb.tp_ffn_workspace_bytes(w.M, w.h, w.f, w.t, dt, tb.MODES[self.mode]), dev)
         self.tb = tb
         return p["X"]
 
@@ -222,11 +281,112 @@ class FFN(Workload):
 
     def config(self):
         w = self.w
-        return {"workload": self.name, "M": w.M, "h": w.h, "f": w.f, "t": w.t, "reduce": self.mode,
-                "w2": "fp16" if self.w2_fp16 else "bf16"}
+        c = {"workload": self.name, "M": w.M, "h": w.h, "f": w.f, "t": w.t, "reduce": self.mode,
+             "dtype": w.dtype}
+        if w.dtype == "bf16":
+            c["w2"] = "fp16 copy of the bf16 W2 (act(Z) in fp16)" if self.w2_fp16 else "bf16"
+        return c
+
+    # -------- oracle
+    def oracle_setup(self, src):
+        """src: dict of input tensors (any device); W1/W2 stay 16-bit on the host and
+        are converted to fp64 chunk by chunk when they are large."""
+        host = {k: v.detach().to("cpu") for k, v in src.items()}
+        big = self.w.h * self.w.f > (1 << 28)
+        st = {"X": _to64(host["X"]), "b1": _to64(host["b1"]), "b2": _to64(host["b2"]), "big": big}
+        if big:
+            st["W1"], st["W2"] = host["W1"], host["W2"]
+        else:
+            st["W1"], st["W2"] = _to64(host["W1"]), _to64(host["W2"])
+        return st
+
+    def oracle_rows(self, st, rng, n):
+        import numpy as np
+        import oracle
+        w = self.w
+        rows = np.sort(rng.choice(w.M, min(n, w.M), replace=False))
+        X = st["X"][rows]
+        if not st["big"]:
+            oracle.ffn_forward(X, st["W1"], st["b1"], st["W2"], st["b2"], X)
+        else:
+            chunks = 16
+            k = w.f // chunks
+
+            def shards():
+                for i in range(chunks):
+                    c = slice(i * k, (i + 1) * k)
+                    yield _to64(st["W1"][:, c]), st["b1"][c], _to64(st["W2"][c, :])
+
+            oracle.ffn_forward_sharded(X, shards(), st["b2"], X)
+        return len(rows), self.flops * len(rows) / w.M
+
+
+class FFNBwd(Workload):
+    """One backward pass of the FFN block (tp_ffn_backward): the input gradient dX and the
+    weight and bias gradients for an upstream gradient dY.  FLOPs: the model count
+    8*M*h*f (dA, dW2, dW1 and dX GEMMs); the call also recomputes step 1 (2*M*h*f more,
+    reported as executed_flops_per_step).  The per-step input is X and dY, stacked."""
+    ref_rows = 8
+
+    def __init__(self, w):
+        self.w = w
+        self.name = "ffn_bwd_" + w.name[len("ffn_"):]
+        self.flops = 2 * w.flops
+        M, h, f, t = w.M, w.h, w.f, w.t
+        self.kernel_amount = {k: ("tensor", 2 * M * h * f, "FLOP") for k in
+                              ("gemm_bwd_recompute", "gemm_bwd_dz", "gemm_bwd_dw2", "gemm_bwd_dw1", "gemm_bwd_dx")}
+        self.kernel_amount["colsum"] = ("hbm", M * f * 2 + M * h * 2, "B")
+
+    def setup(self, dev, rank):
+        import torch
+        from megatron_tensor_transformer_bias_b200 import inputs
+        from megatron_tensor_transformer_bias_b200 import tpblock as tb
+        w = self.w
+        p = inputs.ffn_inputs(w.M, w.h, w.f, "bf16", seed=0, device=dev)
+        g = torch.Generator(device=dev).manual_seed(9000 + 7919 * rank)
+        p["dY"] = torch.randn(w.M, w.h, generator=g, device=dev).to(torch.bfloat16)
+        self.p = p
+        self.W1 = tb.shard_columns(p["W1"], w.t)
+        self.W2 = tb.shard_rows(p["W2"], w.t)
+        self.b1 = tb.shard_vector(p["b1"], w.t)
+        self.dW1 = torch.empty(w.h, w.f, dtype=torch.float32, device=dev)
+        self.dW2 = torch.empty(w.f, w.h, dtype=torch.float32, device=dev)
+        self.db1 = torch.empty(w.f, dtype=torch.float32, device=dev)
+        self.db2 = torch.empty(w.h, dtype=torch.float32, device=dev)
+        self.ws = tb.workspace(tb.tp_ffn_backward_workspace_bytes(w.M, w.h, w.f, w.t), dev)
+        self.tb = tb
+        return torch.stack([p["X"], p["dY"]])
+
+    def make_out(self, X):
+        import torch
+        return torch.empty_like(X[0])
+
+    def step(self, XdY, dX, stream):
+        self.tb.tp_ffn_backward(XdY[0], self.W1, self.b1, self.W2, XdY[1], dX, self.dW1, self.dW2, self.db1,
+                                self.db2, dX_add=XdY[1], ws=self.ws, stream=stream)
+
+    def config(self):
+        w = self.w
+        return {"workload": self.name, "M": w.M, "h": w.h, "f": w.f, "t": w.t, "dtype": "bf16",
+                "gradients": "dX bf16 (+ dY, the residual path); dW1, dW2, db1, db2 fp32 kept on the device",
+                "executed_flops_per_step": 10 * w.M * w.h * w.f, "e2e_io": "X and dY in, dX out"}
+
+    def oracle_setup(self, src):
+        return {k: _to64(v) for k, v in src.items()}
+
+    def oracle_rows(self, st, rng, n):
+        """The oracle's backward on n token rows (their dX rows and their share of dW, db)."""
+        import numpy as np
+        import oracle
+        w = self.w
+        rows = np.sort(rng.choice(w.M, min(n, w.M), replace=False))
+        oracle.ffn_backward(st["X"][rows], st["W1"], st["b1"], st["W2"], st["dY"][rows])
+        return len(rows), self.flops * len(rows) / w.M
 
 
 class Attn(Workload):
+    ref_rows = 8
+
     def __init__(self, w, mode):
         self.w, self.mode = w, mode
         self.name = w.name
@@ -237,6 +397,7 @@ class Attn(Workload):
             "gemm_qkv": ("tensor", 2 * M * h * 3 * H * d, "FLOP"),
             "attention": ("tensor", 4 * B * H * d * pairs, "FLOP"),
             "gemm_row_fused_reduce": ("tensor", 2 * M * H * d * h, "FLOP"),
+            "gemm_row_partials": ("tensor", 2 * M * H * d * h, "FLOP"),
         }
 
     def setup(self, dev, rank):
@@ -244,6 +405,7 @@ class Attn(Workload):
         from megatron_tensor_transformer_bias_b200 import tpblock as tb
         w = self.w
         a = inputs.attn_inputs(w.B, w.S, w.h, w.H, w.d, seed=rank, device=dev)
+        self.p = a
         self.Wqkv = tb.shard_columns(inputs.pack_qkv(a["Wq"], a["Wk"], a["Wv"], w.t, w.H, w.d), w.t)
         self.Wo = tb.shard_rows(a["Wo"], w.t)
         self.bo = a["bo"]
@@ -259,14 +421,31 @@ class Attn(Workload):
     def config(self):
         w = self.w
         return {"workload": self.name, "B": w.B, "S": w.S, "h": w.h, "heads": w.H, "d": w.d, "t": w.t,
-                "causal": w.causal, "reduce": self.mode}
+                "causal": w.causal, "reduce": self.mode, "qkv_p_dtype": "fp16"}
+
+    def oracle_setup(self, src):
+        return {k: _to64(v) for k, v in src.items()}
+
+    def oracle_rows(self, st, rng, n):
+        """n rows of one random sequence; the oracle forms K and V for the whole sequence."""
+        import numpy as np
+        import oracle
+        w = self.w
+        b = int(rng.integers(w.B))
+        rows = b * w.S + np.sort(rng.choice(w.S, min(n, w.S), replace=False))
+        oracle.attn_forward(st["X"], st["Wq"], st["Wk"], st["Wv"], st["Wo"], st["bo"], st["X"], w.B, w.S, w.H,
+                            w.d, w.causal, rows=rows)
+        return len(rows), self.flops * len(rows) / w.M
 
 
 class Layer(Workload):
+    ref_rows = 8
+
     def __init__(self, w, mode):
         self.w, self.mode = w, mode
         self.name = w.name + "_fp16w"
         self.flops = w.flops
+        self.dtype = "bf16 (fp16 weight copies and intermediates)"
         M, h, H, d, B, S, f = w.M, w.h, w.H, w.d, w.B, w.S, w.f
         pairs = S * (S + 1) // 2 if w.causal else S * S
         self.kernel_amount = {
@@ -275,6 +454,7 @@ class Layer(Workload):
             "gemm_column_act": ("tensor", 2 * M * h * f, "FLOP"),
             # two launches per step: the attention out-projection and the FFN row layer (mean per launch)
             "gemm_row_fused_reduce": ("tensor", (2 * M * H * d * h + 2 * M * f * h) // 2, "FLOP"),
+            "gemm_row_partials": ("tensor", (2 * M * H * d * h + 2 * M * f * h) // 2, "FLOP"),
             "layernorm": ("hbm", 5 * M * h, "B"),
         }
 
@@ -306,100 +486,127 @@ class Layer(Workload):
         return {"workload": self.name, "B": w.B, "S": w.S, "h": w.h, "heads": w.H, "d": w.d, "f": w.f, "t": w.t,
                 "causal": w.causal, "reduce": self.mode, "weights": "fp16 copies of the bf16 weights"}
 
+    def oracle_setup(self, src):
+        return {k: _to64(v) for k, v in src.items()}
 
-def make_workload(args):
+    def oracle_rows(self, st, rng, n):
+        """n rows of one random sequence; the oracle takes LN1, K and V over the whole sequence."""
+        import numpy as np
+        import oracle
+        w = self.w
+        b = int(rng.integers(w.B))
+        rows = b * w.S + np.sort(rng.choice(w.S, min(n, w.S), replace=False))
+        oracle.layer_forward(st["X"], st, w.B, w.S, w.H, w.d, eps=w.eps, causal=w.causal, rows=rows)
+        return len(rows), self.flops * len(rows) / w.M
+
+
+def make_workloads(args):
+    """The workloads of this run, the headline last."""
     from megatron_tensor_transformer_bias_b200 import configs
-    if args.workload == "ffn":
-        w = configs.ffn_2048x4096x16384(args.t) if args.t != 4 else configs.HEADLINE
-        return FFN(w, args.mode)
-    if args.workload == "sweep":
-        return FFN(configs.ffn_sweep(args.h, args.t if args.t in configs.SWEEP_SHARDS else 8), args.mode,
-                   w2_fp16=True)
-    if args.workload == "attn":
-        return Attn(configs.ATTN_B2_S2048, args.mode)
-    if args.workload == "layer":
-        return Layer(configs.LAYER_S2048_H8192, args.mode)
-    raise ValueError(args.workload)
+
+    def ffn(t, mode, headline=False):
+        w = configs.ffn_2048x4096x16384(t) if t != 4 else configs.HEADLINE
+        return FFN(w, mode, headline=headline and t == 4 and mode == "fused")
+
+    def sweep(h, t):
+        return FFN(configs.ffn_sweep(h, t), args.mode, w2_fp16=True)
+
+    wl = args.workload
+    if wl == "all":
+        out = [FFN(configs.TINY_FP32_FFN, "partials"), Attn(configs.ATTN_B2_S2048, "fused"),
+               Layer(configs.LAYER_S2048_H8192, "fused")]
+        if args.impl != "reference":   # the oracle's sweep sample needs tens of GB of fp64 weights per step
+            out += [sweep(22528, 1), sweep(22528, 8)]
+        out += [FFNBwd(configs.HEADLINE), ffn(4, "partials"), ffn(4, "fused", headline=True)]
+        return out
+    if wl == "bwd":
+        return [FFNBwd(configs.ffn_2048x4096x16384(args.t) if args.t != 4 else configs.HEADLINE)]
+    if wl == "ffn":
+        return [ffn(args.t, args.mode, headline=True)]
+    if wl == "fp32":
+        return [FFN(configs.TINY_FP32_FFN, "partials")]
+    if wl == "sweep":
+        hs = configs.SWEEP_HIDDEN if args.h == "all" else (int(args.h),)
+        ts = configs.SWEEP_SHARDS if args.t not in configs.SWEEP_SHARDS else (args.t,)
+        return [sweep(h, t) for h in hs for t in ts]
+    if wl == "attn":
+        return [Attn(configs.ATTN_B2_S2048, args.mode)]
+    if wl == "layer":
+        return [Layer(configs.LAYER_S2048_H8192, args.mode)]
+    raise ValueError(wl)
 
 
 # ---------------------------------------------------------------- CPU oracle timing
-def _threads():
-    try:
-        from threadpoolctl import threadpool_info
-        return max(i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas")
-    except Exception:
-        return os.cpu_count()
-
-
-def _oracle_ffn_setup(w, device):
-    import torch
-    from megatron_tensor_transformer_bias_b200 import inputs
-    p = inputs.ffn_inputs(w.M, w.h, w.f, "bf16", seed=0, device=device)
-    return {k: v.to("cpu", dtype=torch.float64).numpy() for k, v in p.items()}
-
-
-def _oracle_ffn_rows(c, rows):
-    import oracle
-    X = c["X"][rows]
-    return oracle.ffn_forward(X, c["W1"], c["b1"], c["W2"], c["b2"], X)
-
-
-def cpu_baseline(w, c, target_s=10.0):
-    """The oracle as it stands, on the FFN workload's token rows, timed on the host cores.
-
-    Repeats whole passes over the M rows (or a single pass over a subset when one pass
-    would take longer) until about `target_s` seconds of CPU work have run."""
+def cpu_baseline(wl, st, target_s=10.0, rows_per_call=64):
+    """The oracle as it stands, timed on the host cores on samples of the workload's
+    token rows until about `target_s` seconds of CPU work have run (at least one call).
+    FLOPs credited per call: rows / M of the workload's algorithmic count."""
     import numpy as np
     rng = np.random.default_rng(0)
-    n0 = min(64, w.M)
+    rows = calls = 0
+    flops = 0.0
     t0 = time.perf_counter()
-    _oracle_ffn_rows(c, np.sort(rng.choice(w.M, n0, replace=False)))
-    per_row = (time.perf_counter() - t0) / n0
-    n = int(min(w.M, max(n0, target_s / max(per_row, 1e-9))))
-    reps = max(1, int(target_s / max(per_row * n, 1e-9)))
-    rows = np.arange(w.M) if n == w.M else np.sort(rng.choice(w.M, n, replace=False))
-    t0 = time.perf_counter()
-    for _ in range(reps):
-        _oracle_ffn_rows(c, rows)
-    dt = time.perf_counter() - t0
-    flops = 4 * n * w.h * w.f * reps
-    return {"value": round(flops / dt / 1e12, 4), "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
-            "sample": f"{reps} pass(es) over {n} of {w.M} token rows of {w.name}, fp64 numpy/OpenBLAS, "
-                      f"{dt:.1f} s wall"}
+    while True:
+        n, fl = wl.oracle_rows(st, rng, rows_per_call)
+        rows += n
+        flops += fl
+        calls += 1
+        dt = time.perf_counter() - t0
+        if dt >= target_s:
+            break
+    out = {"value": round(flops / dt / 1e12, 5), "unit": "TFLOP/s", "kind": "oracle",
+           "sample": f"{calls} oracle call(s) of {min(rows_per_call, wl.w.M)} token rows each ({rows} rows of "
+                     f"{wl.w.M}) of {wl.name}, fp64 numpy/OpenBLAS, {dt:.1f} s wall; credited rows/M of the "
+                     f"workload's FLOPs"}
+    out.update(_host())
+    return out
 
 
-def run_reference(args, wl):
+def run_reference(args, wls):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     import numpy as np
-    w = wl.w if isinstance(wl, FFN) else None
-    if w is None:
-        print(json.dumps({"impl": "reference", "unavailable": "the CPU reference arm covers the FFN workloads"}))
-        return
-    c = _oracle_ffn_setup(w, "cpu")
-    rng = np.random.default_rng(1)
-    rows_per_step = 8
-    for _ in range(args.warmup):
-        _oracle_ffn_rows(c, np.sort(rng.choice(w.M, rows_per_step, replace=False)))
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        _oracle_ffn_rows(c, np.sort(rng.choice(w.M, rows_per_step, replace=False)))
-    dt = time.perf_counter() - t0
-    value = 4 * rows_per_step * w.h * w.f * args.steps / dt / 1e12
-    sample = f"{rows_per_step} of {w.M} token rows of {w.name} per step, fp64 numpy/OpenBLAS"
-    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": wl.config(),
-            "impl": "reference",
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
-                             "sample": sample},
-            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-    print(json.dumps(line), flush=True)
+    from megatron_tensor_transformer_bias_b200 import inputs
+    for wl in wls:
+        w = wl.w
+        if isinstance(wl, FFNBwd):
+            import torch
+            src = inputs.ffn_inputs(w.M, w.h, w.f, "bf16", seed=0, device="cpu")
+            src["dY"] = torch.randn(w.M, w.h, generator=torch.Generator().manual_seed(9000)).to(torch.bfloat16)
+        elif isinstance(wl, FFN):
+            src = inputs.ffn_inputs(w.M, w.h, w.f, w.dtype, seed=0, device="cpu")
+        elif isinstance(wl, Attn):
+            src = inputs.attn_inputs(w.B, w.S, w.h, w.H, w.d, seed=0, device="cpu")
+        else:
+            src = inputs.layer_inputs(w.B, w.S, w.h, w.H, w.d, w.f, seed=0, device="cpu")
+        st = wl.oracle_setup(src)
+        del src
+        rng = np.random.default_rng(1)
+        n = min(wl.ref_rows, w.M)
+        for _ in range(args.warmup):
+            wl.oracle_rows(st, rng, n)
+        flops = 0.0
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            flops += wl.oracle_rows(st, rng, n)[1]
+        dt = time.perf_counter() - t0
+        value = flops / dt / 1e12
+        sample = (f"{n} of {w.M} token rows of {wl.name} per step, fp64 numpy/OpenBLAS; credited rows/M of the "
+                  f"workload's FLOPs")
+        cb = {"value": value, "unit": "TFLOP/s", "kind": "oracle", "sample": sample}
+        cb.update(_host())
+        line = {"metric": wl.metric(), "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": wl.config(),
+                "impl": "reference", "cpu_baseline": cb,
+                "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        del st
 
 
 # ---------------------------------------------------------------- GPU arm
-def run_ours(args, wl):
+def run_ours(args, wls):
     import torch
     import torch.distributed as dist
 
@@ -413,14 +620,26 @@ def run_ours(args, wl):
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    try:
+        tb.lib()
+        for wl in wls:
+            run_one(args, wl, world, rank, local, dev, dist)
+            torch.cuda.empty_cache()
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+def run_one(args, wl, world, rank, local, dev, dist):
+    import torch
+    from megatron_tensor_transformer_bias_b200 import tpblock as tb
 
     def barrier():
         if world > 1:
             dist.barrier()
 
-    tb.lib()
     X = wl.setup(dev, rank)
-    out = torch.empty_like(X)
+    out = wl.make_out(X) if hasattr(wl, "make_out") else torch.empty_like(X)
     stream = torch.cuda.current_stream()
 
     def step():
@@ -429,7 +648,7 @@ def run_ours(args, wl):
     for _ in range(args.warmup):
         step()
     if tb.tp_get_device_status(stream) != tb.TP_OK:
-        raise RuntimeError("device status after warm-up: " + tb.last_error())
+        raise RuntimeError(f"{wl.name}: device status after warm-up: " + tb.last_error())
 
     def timed(fn, k):
         barrier()
@@ -483,7 +702,22 @@ def run_ours(args, wl):
         torch.cuda.synchronize()
         ms_e2e = timed(step_e2e, args.steps)
     if tb.tp_get_device_status(stream) != tb.TP_OK:
-        raise RuntimeError("device status after timing: " + tb.last_error())
+        raise RuntimeError(f"{wl.name}: device status after timing: " + tb.last_error())
+
+    # sustained: the same step looped for >= 2 s (under the power cap), timed the same way
+    sustained = None
+    if getattr(wl, "headline", False) and not args.no_sustained:
+        k_s = max(args.steps, int(2.2 / max(ms * 1e-3 / args.steps, 1e-6)))
+        with ClockSampler(local, period_s=0.05) as clk_s:
+            ms_s = timed(lambda i: step(), k_s)
+        if tb.tp_get_device_status(stream) != tb.TP_OK:
+            raise RuntimeError(f"{wl.name}: device status after the sustained loop: " + tb.last_error())
+        v_s = wl.flops * world / (ms_s * 1e-3 / k_s) / 1e12
+        peaks = _peaks()
+        sustained = {"value": round(v_s, 2), "unit": "TFLOP/s", "steps": k_s, "seconds": round(ms_s / 1e3, 3),
+                     "ms_per_step": ms_s / k_s, "peak": peaks["bf16_tflops_sustained"],
+                     "frac_of_sustained_peak": round(v_s / world / peaks["bf16_tflops_sustained"], 4),
+                     "pct_of_nominal_2250": round(100 * v_s / world / 2250.0, 2), "clocks": clk_s.summary()}
 
     per = {}
     for name, kms in recs:
@@ -495,49 +729,54 @@ def run_ours(args, wl):
     dom_avg_ms = per[dominant][1] / per[dominant][0]
     bound, amount, unit = wl.kernel_amount.get(dominant, ("tensor", 0, "FLOP"))
     peaks = _peaks()
-    sustained = ms > 2000.0
+    long_run = ms > 2000.0
     if bound == "hbm":
         peak, punit, achieved = peaks["hbm_gbs"], "GB/s", amount / (dom_avg_ms * 1e-3) / 1e9
         pkind = "measured copy" if peaks["source"] == "measured" else "fallback"
-    else:
-        peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    elif bound == "alu":
+        # fp32 FFMA on the CUDA cores: 148 SMs x 128 lanes x 2 FLOP per clock at the maximum SM clock
+        peak = 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
         punit, achieved = "TFLOP/s", amount / (dom_avg_ms * 1e-3) / 1e12
-        pkind = ("sustained" if sustained else "burst") + " bf16, " + peaks["source"]
+        pkind = "fp32 FFMA, 148 SMs x 128 lanes x 2 FLOP x max SM clock"
+    else:
+        peak = peaks["bf16_tflops_sustained"] if long_run else peaks["bf16_tflops"]
+        punit, achieved = "TFLOP/s", amount / (dom_avg_ms * 1e-3) / 1e12
+        pkind = ("sustained" if long_run else "burst") + " bf16, " + peaks["source"]
     value = wl.flops * world / (ms * 1e-3 / args.steps) / 1e12
 
     if rank == 0:
         line = {
-            "metric": METRIC if isinstance(wl, FFN) and wl.w.t == 4 and wl.w.M == 2048 and wl.w.h == 4096
-            else f"TFLOP/s, {wl.name}, 1 B200",
-            "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "metric": wl.metric(),
+            "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16" if not isinstance(wl, Layer) else "bf16/f16",
-            "data": "synthetic (seeded randn; X~N(0,1), W~N(0,0.02^2), b~N(0,0.01^2), residual=X)",
+            "vs_baseline": None, "dtype": wl.dtype, "data": DATA,
             "config": dict(wl.config(), parallelism=f"replicas x{world}" if world > 1
                            else "single GPU, t logical shards",
-                           l2="per-step operands exceed the 126 MB L2, no flush"),
+                           l2="per-step operands exceed the 126 MB L2, no flush" if wl.flops > 1e11
+                           else "operands fit in L2 (launch-bound workload)"),
             "pct_of_peak": {"nominal_2250": round(100 * value / world / 2250.0, 2),
-                            "measured_burst": round(100 * value / world / peaks["bf16_tflops"], 2),
-                            "measured_sustained": round(100 * value / world / peaks["bf16_tflops_sustained"], 2)},
-            "roofline": {"kernel": dominant, "bound": bound, "achieved": round(achieved, 2), "peak": peak,
+                            "measured_burst": round(100 * value / world / peaks["bf16_tflops"], 2)},
+            "roofline": {"kernel": dominant, "bound": bound, "achieved": round(achieved, 3), "peak": round(peak, 1),
                          "unit": punit, "frac": round(achieved / peak, 4), "peak_kind": pkind,
                          "traffic": _traffic(wl.name, dominant), "amount_per_launch": amount,
                          "amount_unit": unit, "avg_launch_ms": dom_avg_ms},
             "kernels": {k: {"launches": v[0], "total_ms": round(v[1], 3), "share": round(v[1] / ms_traced, 4)}
                         for k, v in per.items()},
-            "e2e": {"value": round(wl.flops * world / (ms_e2e * 1e-3 / args.steps) / 1e12, 2), "unit": "TFLOP/s",
+            "e2e": {"value": round(wl.flops * world / (ms_e2e * 1e-3 / args.steps) / 1e12, 3), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": X.numel() * X.element_size(),
                     "d2h_bytes_per_step": out.numel() * out.element_size(),
                     "pipeline": "H2D, compute, D2H on three streams, double-buffered"},
             "gpu_launches": launches,
             "clocks": clk.summary(),
         }
-        if world == 1 and not args.no_cpu_baseline and isinstance(wl, FFN):
-            c = _oracle_ffn_setup(wl.w, dev)
-            line["cpu_baseline"] = cpu_baseline(wl.w, c)
+        if sustained:
+            line["sustained"] = sustained
+        if world == 1 and not args.no_cpu_baseline:
+            st = wl.oracle_setup(wl.p)
+            line["cpu_baseline"] = cpu_baseline(wl, st, target_s=args.cpu_seconds)
+            del st
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    barrier()
 
 
 def main():
@@ -546,19 +785,21 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["ffn", "attn", "layer", "sweep"], default="ffn")
+    ap.add_argument("--workload", choices=["all", "ffn", "bwd", "attn", "layer", "sweep", "fp32"], default="all")
     ap.add_argument("--t", type=int, default=4)
-    ap.add_argument("--h", type=int, default=22528)
+    ap.add_argument("--h", default="22528", help="sweep hidden size, or 'all'")
     ap.add_argument("--mode", choices=["fused", "partials"], default="fused")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-sustained", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    wl = make_workload(args)
+    wls = make_workloads(args)
     if args.impl == "reference":
-        run_reference(args, wl)
+        run_reference(args, wls)
     else:
-        run_ours(args, wl)
+        run_ours(args, wls)
 
 
 if __name__ == "__main__":

@@ -1,6 +1,7 @@
 /*
- * libtpblock -- the Megatron column->row tensor-parallel transformer block,
- * forward pass, on one B200 (sm_100a).
+ * libtpblock -- the Megatron column->row tensor-parallel transformer block on
+ * one B200 (sm_100a): forward passes of the FFN block, the attention sub-layer
+ * and the pre-LN layer, and the backward pass of the FFN block.
  *
  * Source of the method: "Tensor Parallelism > Combining Column and Row
  * Parallelism" (mbrenndoerfer.com), cited below as [TP-CR]:
@@ -62,7 +63,8 @@ typedef enum {
   TP_ERR_UNSUPPORTED = 2, /* valid but outside what the kernels implement */
   TP_ERR_WORKSPACE = 3,   /* workspace missing or smaller than *_workspace_bytes */
   TP_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
-  TP_ERR_TIMEOUT = 5      /* a device wait ran out (reported by tp_get_device_status) */
+  TP_ERR_TIMEOUT = 5,     /* a device wait ran out (reported by tp_get_device_status) */
+  TP_ERR_RANGE = 6        /* an fp16 intermediate exceeded 65504 (reported by tp_get_device_status) */
 } tp_status;
 
 typedef enum { TP_BF16 = 0, TP_FP32 = 1, TP_FP16 = 2 } tp_dtype;
@@ -74,9 +76,19 @@ typedef enum { TP_BF16 = 0, TP_FP32 = 1, TP_FP16 = 2 } tp_dtype;
  *                     (ascending or descending K, whichever starts on data
  *                     still in L2), and its epilogue adds the bias and the
  *                     residual.  The result is the same bits for every t.
+ *                     A tile's place in the schedule depends on the number
+ *                     of CTA pairs the device runs at once (74 on a 148-SM
+ *                     B200), so the bits are reproducible across runs and
+ *                     processes on devices with the same SM count.
  * TP_REDUCE_PARTIALS: the row GEMM writes t fp32 partials Y_i [t, M, h] to the
- *                     workspace; a reduce kernel sums them in order 0..t-1
- *                     and adds bias and residual. */
+ *                     workspace.  Inside the same kernel, the shard that is the
+ *                     last to finish a 32-row x 128-column region of the
+ *                     output sums that region's t partials in the order
+ *                     0..t-1 and adds bias and residual, so the reduction
+ *                     runs while other tiles are still being multiplied
+ *                     ([TP-CR] step 3 overlapped with step 2).  The sums are
+ *                     the ones a separate pass over the partials would take:
+ *                     same order, same bits. */
 typedef enum { TP_REDUCE_FUSED = 0, TP_REDUCE_PARTIALS = 1 } tp_reduce_mode;
 
 /* Element-wise nonlinearity of step 1: exact GeLU z*Phi(z) (erf form) or ReLU. */
@@ -87,7 +99,10 @@ typedef enum { TP_ACT_GELU = 0, TP_ACT_RELU = 1 } tp_activation;
  * GEMM the activation operand is produced in its weight's type: an fp16 W2
  * makes act(Z) fp16, an fp16 Wqkv makes the layer's LN1 output fp16, and so on.
  * fp16 has 3 more mantissa bits than bf16 at the same tensor-core rate, and
- * bf16 weights of ordinary magnitude convert to fp16 exactly. */
+ * bf16 weights of ordinary magnitude convert to fp16 exactly; a bf16 caller
+ * gets fp16 intermediates only by passing fp16 copies of its weights.  fp16's
+ * range ends at 65504: an intermediate above it is stored as +-inf and
+ * tp_get_device_status() reports TP_ERR_RANGE. */
 typedef struct {
   const void* ptr; /* device pointer to element (0, 0) of the shard */
   int64_t ld;      /* row stride in elements */
@@ -111,8 +126,10 @@ typedef void* tp_stream_t; /* cudaStream_t */
  *  dtype    TP_BF16 (tensor cores) or TP_FP32 (exact fp32 FFMA, no TF32).
  *  mode     see tp_reduce_mode (ignored for TP_FP32, which always uses partials).
  *  ws       device workspace of at least tp_ffn_workspace_bytes(...) bytes,
- *           256-byte aligned.  Holds act(Z) [M, f] (and the partials in
- *           TP_REDUCE_PARTIALS mode).  Its contents on entry are ignored.
+ *           256-byte aligned.  Holds act(Z) [M, f] (and, in TP_REDUCE_PARTIALS
+ *           mode, the partials and one arrival counter per 32x128 output region,
+ *           which the call zeroes on the stream first).  Its contents on entry
+ *           are ignored.
  * Limits: 1 <= t <= TP_MAX_SHARDS, f % t == 0, M >= 1.
  */
 TP_API size_t tp_ffn_workspace_bytes(int64_t M, int64_t h, int64_t f, int t, tp_dtype dtype, tp_reduce_mode mode);
@@ -140,11 +157,55 @@ TP_API tp_status tp_ffn_forward_act(const void* X, int64_t M, int64_t h, int64_t
  * or cudaFree.  Every call on a device shares that array, so calls that overlap
  * on the GPU (e.g. on two streams) race; nothing in it needs to start at zero.
  * The first call on each device looks up the array's device address: make it
- * before any stream capture.  Each GPU that loads the library keeps the 16 MiB
- * until the process exits. */
+ * before any stream capture.  Later calls on a stream that is not capturing
+ * look it up again (a device reset may move it); capturing calls reuse the
+ * last address.  Each GPU that loads the library keeps the 16 MiB until the
+ * process exits. */
 TP_API tp_status tp_ffn_forward_noalloc(const void* X, int64_t M, int64_t h, int64_t f, int t, const tp_shard* W1,
                                         const void* const* b1, const tp_shard* W2, const void* b2,
                                         const void* residual, void* out, tp_stream_t stream);
+
+/* ------------------------------------------------------------------ FFN block, backward pass
+ * Gradients of the FFN block for the upstream gradient dY = dL/d(out).  [TP-CR]
+ * gives the forward pass and its one all-reduce per two-layer block; the
+ * backward pass is the chain rule back through steps 3, 2 and 1, read with the
+ * page's column/row pairing: dY is the same for every shard (it is the
+ * gradient of the all-reduce's output), so the row layer's input gradient
+ * dA_i = dY W2_i^T is local to shard i, and the column layer's input gradient
+ * dX = sum_i dZ_i W1_i^T is a sum over shards, the backward pass's one
+ * reduction (taken here in one accumulator over the shards' K-slices).
+ *
+ *   Z_i = X W1_i + b1_i,  A_i = act(Z_i)       (recomputed from X: nothing is
+ *                                               kept from the forward call)
+ *   dW2_i = A_i^T dY,     db2 = column sums of dY
+ *   dZ_i = (dY W2_i^T) * act'(Z_i)
+ *   dW1_i = X^T dZ_i,     db1_i = column sums of dZ_i
+ *   dX = sum_i dZ_i W1_i^T (+ dX_add)
+ *
+ *  X, W1, b1, W2  as in tp_ffn_forward, bf16 only (TP_BF16 shards).
+ *  dY       [M, h] bf16, contiguous.
+ *  dX_add   [M, h] bf16 or NULL: added to dX (pass dY when the forward's
+ *           residual was X: the residual path's gradient is dY itself).
+ *  dX       [M, h] bf16 out, contiguous; must not alias X, dY or dX_add.
+ *  dW1      [h, f] fp32 out, contiguous: shard i's gradient is the column
+ *           block [i*f/t, (i+1)*f/t).  Overwritten, not accumulated.
+ *  db1      [f] fp32 out or NULL.   dW2  [f, h] fp32 out, contiguous: shard
+ *           i's gradient is the row block [i*f/t, (i+1)*f/t).  db2 [h] fp32
+ *           out or NULL.
+ *  act      the forward's nonlinearity (GeLU'(z) = Phi(z) + z phi(z); ReLU'
+ *           is 1 for z > 0, else 0).
+ *  ws       tp_ffn_backward_workspace_bytes(...) bytes, 256-byte aligned:
+ *           act(Z) (bf16), act'(Z) (fp16, in [-0.17, 1.13] for GeLU) and dZ
+ *           (bf16), each [M, f], and the column sums' scratch.
+ * The sums over rows (dW, db) and over shards (dX) are taken in a fixed
+ * order: results are bitwise reproducible on devices with the same SM count.
+ * M == 0 zeroes dW1, dW2, db1, db2.  Limits as tp_ffn_forward's bf16 path.
+ */
+TP_API size_t tp_ffn_backward_workspace_bytes(int64_t M, int64_t h, int64_t f, int t);
+TP_API tp_status tp_ffn_backward(const void* X, int64_t M, int64_t h, int64_t f, int t, const tp_shard* W1,
+                                 const void* const* b1, const tp_shard* W2, const void* dY, const void* dX_add,
+                                 void* dX, float* dW1, float* db1, float* dW2, float* db2, tp_activation act,
+                                 void* ws, size_t ws_bytes, tp_stream_t stream);
 
 /* ------------------------------------------------------------------ parallel linears
  * Column-parallel linear alone ([TP-CR] step 1), bf16 or fp16 (W's dtype):
@@ -232,7 +293,14 @@ TP_API tp_status tp_reduce_partials(const float* P, int t, int64_t M, int64_t h,
 /* ------------------------------------------------------------------ status, limits, tracing */
 /* Synchronise `stream`, then read and clear the device status word of the
  * current device.  TP_ERR_TIMEOUT if a device wait ran out since the last call;
- * TP_ERR_CUDA if the synchronisation itself failed. */
+ * else TP_ERR_RANGE if a value that a kernel stored in an fp16 intermediate
+ * (act(Z) of an fp16 W2, Q/K/V, O of an fp16 Wo, a LayerNorm output of an fp16
+ * weight) had a magnitude above 65504, the largest fp16 number: such a value is
+ * stored as +-inf, and tp_last_error() names the intermediate.  The check costs
+ * one max per stored value and never stops a kernel.  bf16 intermediates have
+ * fp32's range and are not checked.  TP_ERR_CUDA if the synchronisation itself
+ * failed.  The status word's address is looked up once per device; resetting a
+ * device (cudaDeviceReset) that the library has used is not supported. */
 TP_API tp_status tp_get_device_status(tp_stream_t stream);
 
 /* Time limit of every device-side wait, in nanoseconds (default 2e9). */

@@ -20,7 +20,10 @@ __device__ uint32_t g_status_word;
 namespace {
 constexpr int MAX_DEV = 64;
 int g_sm_count[MAX_DEV] = {0};
-uint32_t* g_status_ptr[MAX_DEV] = {nullptr};
+// Device address of g_status_word per device, looked up once.  A cudaDeviceReset
+// unloads the module, so the cached address is stale after one: the library does not
+// support resetting a device it has used.
+std::atomic<uint32_t*> g_status_ptr[MAX_DEV];
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
 thread_local std::string t_last_error;
 
@@ -76,12 +79,14 @@ int sm_count() {
 uint32_t* device_status_ptr() {
   const int d = current_device();
   if (d < 0 || d >= MAX_DEV) return nullptr;
-  if (!g_status_ptr[d]) {
+  uint32_t* cached = g_status_ptr[d].load();
+  if (!cached) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
-    g_status_ptr[d] = static_cast<uint32_t*>(p);
+    cached = static_cast<uint32_t*>(p);
+    g_status_ptr[d].store(cached);
   }
-  return g_status_ptr[d];
+  return cached;
 }
 
 uint64_t wait_limit_ns() { return g_wait_limit_ns.load(); }
@@ -146,6 +151,22 @@ tp_status make_tmap_2d(CUtensorMap* map, const void* base, int f16, uint64_t inn
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return TP_OK;
+}
+
+tp_status make_tmap_mn(CUtensorMap* map, const void* base, int f16, uint64_t mn_cols, uint64_t k_rows,
+                       uint64_t row_stride_bytes) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  // [k_rows, mn_cols] row-major seen as (64 columns of a block, k_rows, mn_cols / 64 blocks)
+  cuuint64_t dims[3] = {64, k_rows, mn_cols / 64};
+  cuuint64_t strides[2] = {row_stride_bytes, 128};
+  cuuint32_t box[3] = {64, 64, 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled(mn) failed (%d)", static_cast<int>(r));
   return TP_OK;
 }
 
@@ -234,10 +255,41 @@ inline int is_f16(const tp_shard* W) { return W[0].dtype == TP_FP16 ? 1 : 0; }
     if (_s != TP_OK) return _s;        \
   } while (0)
 
+// ---------------------------------------------------------------- partials-mode workspace
+// The row GEMM's fp32 partials [t, M, n], then the arrival counters of the in-epilogue
+// reduction (one 32-bit word per 32-row x 128-column region of the output).
+size_t row_partials_ws(int64_t M, int64_t n, int t) {
+  return align_up(static_cast<size_t>(t) * M * n * 4) + align_up(partial_counter_count(M, n) * 4);
+}
+uint32_t* row_partials_counters(float* P, int64_t M, int64_t n, int t) {
+  return reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(P) + align_up(static_cast<size_t>(t) * M * n * 4));
+}
+
+// The separate reduce kernel instead of the reduction in the row GEMM's epilogue
+// (TPB_SEPARATE_REDUCE=1; the same sums in the same order).
+bool separate_reduce() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("TPB_SEPARATE_REDUCE");
+    v = (e && e[0] == '1') ? 1 : 0;
+  }
+  return v == 1;
+}
+
+// Zero the arrival counters of a partials-mode row GEMM (before the sub-layer's first
+// launch, so that its kernels stay chained by programmatic dependent launch).
+tp_status zero_row_counters(float* P, int64_t M, int64_t n, int t, cudaStream_t stream) {
+  if (separate_reduce()) return TP_OK;
+  const cudaError_t e =
+      cudaMemsetAsync(row_partials_counters(P, M, n, t), 0, partial_counter_count(M, n) * 4, stream);
+  if (e != cudaSuccess) return fail(TP_ERR_CUDA, "cudaMemsetAsync of the reduction counters: %s", cudaGetErrorString(e));
+  return TP_OK;
+}
+
 // ---------------------------------------------------------------- FFN (bf16)
 size_t ffn_bf16_ws(int64_t M, int64_t h, int64_t f, int t, tp_reduce_mode mode) {
   size_t s = align_up(static_cast<size_t>(M) * f * 2);
-  if (mode == TP_REDUCE_PARTIALS) s += align_up(static_cast<size_t>(t) * M * h * 4);
+  if (mode == TP_REDUCE_PARTIALS) s += row_partials_ws(M, h, t);
   return s;
 }
 
@@ -261,7 +313,7 @@ tp_status run_column(const void* X, int64_t M, int64_t k, int64_t ncol, int t, c
   memset(&a, 0, sizeof(a));
   const int f16 = is_f16(W);
   TP_TRY(make_tmap_2d(&a.tmA, X, f16, k, M, k * 2, 64, GEMM_BM));
-  for (int i = 0; i < t; ++i) TP_TRY(make_tmap_2d(&a.tmB[i], W[i].ptr, f16, ncol, k, W[i].ld * 2, 64, 64));
+  for (int i = 0; i < t; ++i) TP_TRY(make_tmap_mn(&a.tmB[i], W[i].ptr, f16, ncol, k, W[i].ld * 2));
   a.M = static_cast<int>(M); a.N = static_cast<int>(ncol); a.Kg = static_cast<int>(k); a.G = t;
   a.concat = 0; a.a_k_per_group = 0;
   a.epi = EPI_ACT; a.act = act; a.ab_f16 = f16;
@@ -284,7 +336,7 @@ tp_status run_row(const void* A, int64_t M, int64_t kg, int64_t n, int t, const 
   memset(&a, 0, sizeof(a));
   const int f16 = is_f16(W);
   TP_TRY(make_tmap_2d(&a.tmA, A, f16, kg * t, M, kg * t * 2, 64, GEMM_BM));
-  for (int i = 0; i < t; ++i) TP_TRY(make_tmap_2d(&a.tmB[i], W[i].ptr, f16, n, kg, W[i].ld * 2, 64, 64));
+  for (int i = 0; i < t; ++i) TP_TRY(make_tmap_mn(&a.tmB[i], W[i].ptr, f16, n, kg, W[i].ld * 2));
   a.ab_f16 = f16;
   a.M = static_cast<int>(M); a.N = static_cast<int>(n); a.Kg = static_cast<int>(kg); a.G = t;
   a.a_k_per_group = static_cast<int>(kg);
@@ -303,8 +355,17 @@ tp_status run_row(const void* A, int64_t M, int64_t kg, int64_t n, int t, const 
   a.concat = 0;
   a.epi = EPI_PARTIAL_F32;
   a.out = P; a.ld_out = n; a.out_group_stride = M * n;
-  TP_TRY(launch_gemm(a, stream, "gemm_row_partials"));
-  return launch_reduce_partials(P, t, M, n, bias, 0, resid, resid_fp32, out, out_fp32, stream);
+  if (separate_reduce()) {
+    TP_TRY(launch_gemm(a, stream, "gemm_row_partials"));
+    return launch_reduce_partials(P, t, M, n, bias, 0, resid, resid_fp32, out, out_fp32, stream);
+  }
+  // step 3 in the epilogue of the last shard's tiles: partials 0..t-2 are stored, the last
+  // one is added to them straight from the accumulator, in the order 0..t-1
+  a.counters = row_partials_counters(P, M, n, t);
+  a.red_out = out; a.red_out_f32 = out_fp32;
+  if (!out_fp32) TP_TRY(make_tmap_out(&a.tmOut, out, 0, static_cast<uint64_t>(n), M, n * 2));
+  a.bias = bias; a.resid = resid; a.ld_resid = n; a.resid_fp32 = resid_fp32;
+  return launch_gemm(a, stream, "gemm_row_partials");
 }
 
 // X has W1's dtype; act(Z) is stored in W2's dtype.
@@ -315,6 +376,7 @@ tp_status ffn_bf16(const void* X, int64_t M, int64_t h, int64_t f, int t, const 
   const int64_t fs = f / t;
   uint16_t* Zh = static_cast<uint16_t*>(ws);
   float* P = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align_up(static_cast<size_t>(M) * f * 2));
+  if (mode == TP_REDUCE_PARTIALS) TP_TRY(zero_row_counters(P, M, h, t, stream));
   TP_TRY(run_column(X, M, h, fs, t, W1, b1, act, Zh, is_f16(W2) ? OUT_F16 : OUT_BF16, f, stream));
   return run_row(Zh, M, fs, h, t, W2, b2, resid, resid_fp32, out, out_fp32, mode, P, stream);
 }
@@ -354,6 +416,108 @@ tp_status validate_ffn(const void* X, int64_t M, int64_t h, int64_t f, int t, co
   return TP_OK;
 }
 
+// ---------------------------------------------------------------- FFN backward (bf16)
+// Workspace: act(Z) [M, f] bf16 | act'(Z) [M, f] fp16 | dZ [M, f] bf16 | column-sum scratch.
+struct FfnBwdWs {
+  uint16_t *A, *G, *dZ;
+  float* part;
+};
+
+size_t ffn_bwd_ws_bytes(int64_t M, int64_t h, int64_t f) {
+  const size_t mf = align_up(static_cast<size_t>(M) * f * 2);
+  return 3 * mf + align_up(colsum_workspace_bytes(M, f > h ? f : h));
+}
+
+FfnBwdWs ffn_bwd_ws_layout(void* ws, int64_t M, int64_t f) {
+  const size_t mf = align_up(static_cast<size_t>(M) * f * 2);
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  return {reinterpret_cast<uint16_t*>(p), reinterpret_cast<uint16_t*>(p + mf), reinterpret_cast<uint16_t*>(p + 2 * mf),
+          reinterpret_cast<float*>(p + 3 * mf)};
+}
+
+tp_status ffn_backward_bf16(const void* X, int64_t M, int64_t h, int64_t f, int t, const tp_shard* W1,
+                            const void* const* b1, const tp_shard* W2, const void* dY, const void* dX_add, void* dX,
+                            float* dW1, float* db1, float* dW2, float* db2, int act, void* ws, cudaStream_t stream) {
+  const int64_t fs = f / t;
+  FfnBwdWs w = ffn_bwd_ws_layout(ws, M, f);
+  uint32_t* status = device_status_ptr();
+  const uint64_t lim = wait_limit_ns();
+  // 1. recompute step 1: act(Z_i) (bf16) and act'(Z_i) (fp16), Z_i = X W1_i + b1_i
+  {
+    GemmArgs a;
+    memset(&a, 0, sizeof(a));
+    TP_TRY(make_tmap_2d(&a.tmA, X, 0, h, M, h * 2, 64, GEMM_BM));
+    for (int i = 0; i < t; ++i) TP_TRY(make_tmap_mn(&a.tmB[i], W1[i].ptr, 0, fs, h, W1[i].ld * 2));
+    TP_TRY(make_tmap_out(&a.tmOut, w.A, 0, static_cast<uint64_t>(f), M, f * 2));
+    TP_TRY(make_tmap_out(&a.tmOut2, w.G, 1, static_cast<uint64_t>(f), M, f * 2));
+    a.M = static_cast<int>(M); a.N = static_cast<int>(fs); a.Kg = static_cast<int>(h); a.G = t;
+    a.epi = EPI_ACT_GRAD; a.act = act;
+    a.out = w.A; a.ld_out = f; a.out_col_per_group = fs; a.out_type = OUT_BF16; a.tma_store = 1;
+    for (int i = 0; i < t; ++i) a.bias_g[i] = b1 ? b1[i] : nullptr;
+    a.status = status; a.wait_limit_ns = lim;
+    TP_TRY(launch_gemm(a, stream, "gemm_bwd_recompute"));
+  }
+  // 2. dZ_i = (dY W2_i^T) * act'(Z_i): the row layer's input gradient is local to each shard
+  {
+    GemmArgs a;
+    memset(&a, 0, sizeof(a));
+    TP_TRY(make_tmap_2d(&a.tmA, dY, 0, h, M, h * 2, 64, GEMM_BM));
+    for (int i = 0; i < t; ++i) TP_TRY(make_tmap_2d(&a.tmB[i], W2[i].ptr, 0, h, fs, W2[i].ld * 2, 64, 128));
+    TP_TRY(make_tmap_out(&a.tmOut, w.dZ, 0, static_cast<uint64_t>(f), M, f * 2));
+    a.M = static_cast<int>(M); a.N = static_cast<int>(fs); a.Kg = static_cast<int>(h); a.G = t;
+    a.b_kmajor = 1;
+    a.epi = EPI_MUL_GRAD; a.grad_mul = w.G; a.ld_grad = f;
+    a.out = w.dZ; a.ld_out = f; a.out_col_per_group = fs; a.out_type = OUT_BF16; a.tma_store = 1;
+    a.status = status; a.wait_limit_ns = lim;
+    TP_TRY(launch_gemm(a, stream, "gemm_bwd_dz"));
+  }
+  // 3. dW2_i = act(Z_i)^T dY (rows i*f/t.. of dW2)
+  {
+    GemmArgs a;
+    memset(&a, 0, sizeof(a));
+    TP_TRY(make_tmap_mn(&a.tmA, w.A, 0, f, M, f * 2));
+    for (int i = 0; i < t; ++i) TP_TRY(make_tmap_mn(&a.tmB[i], dY, 0, h, M, h * 2));
+    a.M = static_cast<int>(fs); a.N = static_cast<int>(h); a.Kg = static_cast<int>(M); a.G = t;
+    a.a_mn = 1; a.a_m_per_group = static_cast<int>(fs);
+    a.epi = EPI_PARTIAL_F32;
+    a.out = dW2; a.ld_out = h; a.out_group_stride = fs * h;
+    a.status = status; a.wait_limit_ns = lim;
+    TP_TRY(launch_gemm(a, stream, "gemm_bwd_dw2"));
+  }
+  // 4. dW1_i = X^T dZ_i (columns i*f/t.. of dW1)
+  {
+    GemmArgs a;
+    memset(&a, 0, sizeof(a));
+    TP_TRY(make_tmap_mn(&a.tmA, X, 0, h, M, h * 2));
+    for (int i = 0; i < t; ++i) TP_TRY(make_tmap_mn(&a.tmB[i], w.dZ + i * fs, 0, fs, M, f * 2));
+    a.M = static_cast<int>(h); a.N = static_cast<int>(fs); a.Kg = static_cast<int>(M); a.G = t;
+    a.a_mn = 1; a.a_m_per_group = 0;
+    a.epi = EPI_PARTIAL_F32;
+    a.out = dW1; a.ld_out = f; a.out_group_stride = fs;
+    a.status = status; a.wait_limit_ns = lim;
+    TP_TRY(launch_gemm(a, stream, "gemm_bwd_dw1"));
+  }
+  // 5. dX = sum_i dZ_i W1_i^T (+ dX_add): the column layer's input gradient is the sum over
+  //    shards -- the backward pass's reduction, taken in one accumulator over the shards' K-slices
+  {
+    GemmArgs a;
+    memset(&a, 0, sizeof(a));
+    TP_TRY(make_tmap_2d(&a.tmA, w.dZ, 0, f, M, f * 2, 64, GEMM_BM));
+    for (int i = 0; i < t; ++i) TP_TRY(make_tmap_2d(&a.tmB[i], W1[i].ptr, 0, fs, h, W1[i].ld * 2, 64, 128));
+    TP_TRY(make_tmap_out(&a.tmOut, dX, 0, static_cast<uint64_t>(h), M, h * 2));
+    a.M = static_cast<int>(M); a.N = static_cast<int>(h); a.Kg = static_cast<int>(fs); a.G = t;
+    a.concat = 1; a.a_k_per_group = static_cast<int>(fs); a.b_kmajor = 1;
+    a.epi = EPI_BIAS_RESID; a.bias = nullptr; a.resid = dX_add; a.ld_resid = h; a.resid_fp32 = 0;
+    a.out = dX; a.ld_out = h; a.out_type = OUT_BF16; a.tma_store = 1;
+    a.status = status; a.wait_limit_ns = lim;
+    TP_TRY(launch_gemm(a, stream, "gemm_bwd_dx"));
+  }
+  // 6. bias gradients: column sums of dZ and dY in a fixed order
+  if (db1) TP_TRY(launch_colsum(w.dZ, M, f, f, w.part, db1, stream));
+  if (db2) TP_TRY(launch_colsum(dY, M, h, h, w.part, db2, stream));
+  return TP_OK;
+}
+
 // ---------------------------------------------------------------- attention (bf16)
 struct AttnWs {
   uint16_t *q, *k, *v, *o;
@@ -363,7 +527,7 @@ struct AttnWs {
 size_t attn_ws_bytes_i(int64_t B, int64_t S, int64_t h, int64_t H, int64_t d, int t, tp_reduce_mode mode) {
   const size_t qkv = align_up(static_cast<size_t>(B) * S * H * d * 2);
   size_t s = 4 * qkv;
-  if (mode == TP_REDUCE_PARTIALS) s += align_up(static_cast<size_t>(t) * B * S * h * 4);
+  if (mode == TP_REDUCE_PARTIALS) s += row_partials_ws(B * S, h, t);
   return s;
 }
 
@@ -398,6 +562,7 @@ tp_status attn_bf16(const void* X, int B, int S, int h, int H, int d, int t, con
   const int Hg = H / t;
   const int64_t ncol = 3LL * Hg * d;
   AttnWs w = attn_ws_layout(ws, B, S, H, d);
+  if (mode == TP_REDUCE_PARTIALS) TP_TRY(zero_row_counters(w.P, M, h, t, stream));
   // QKV projection, column-parallel by head group, scattered to [B, H, S, d].
   {
     GemmArgs a;
@@ -405,7 +570,7 @@ tp_status attn_bf16(const void* X, int B, int S, int h, int H, int d, int t, con
     const int f16 = is_f16(Wqkv);  // X has Wqkv's dtype
     TP_TRY(make_tmap_2d(&a.tmA, X, f16, h, M, static_cast<uint64_t>(h) * 2, 64, GEMM_BM));
     for (int i = 0; i < t; ++i)
-      TP_TRY(make_tmap_2d(&a.tmB[i], Wqkv[i].ptr, f16, ncol, h, Wqkv[i].ld * 2, 64, 64));
+      TP_TRY(make_tmap_mn(&a.tmB[i], Wqkv[i].ptr, f16, ncol, h, Wqkv[i].ld * 2));
     a.ab_f16 = f16;
     a.M = static_cast<int>(M); a.N = static_cast<int>(ncol); a.Kg = h; a.G = t;
     a.concat = 0; a.a_k_per_group = 0;
@@ -507,7 +672,7 @@ tp_status tp_column_linear_forward(const void* X, int64_t M, int64_t k, int64_t 
 
 size_t tp_row_linear_workspace_bytes(int64_t M, int64_t n, int t, tp_reduce_mode mode) {
   if (mode != TP_REDUCE_PARTIALS || M <= 0 || n <= 0 || t < 1) return 0;
-  return align_up(static_cast<size_t>(t) * M * n * 4);
+  return row_partials_ws(M, n, t);
 }
 
 tp_status tp_row_linear_forward(const void* A, int64_t M, int64_t k, int64_t n, int t, const tp_shard* W,
@@ -526,8 +691,57 @@ tp_status tp_row_linear_forward(const void* A, int64_t M, int64_t k, int64_t n, 
   const size_t need = tp_row_linear_workspace_bytes(M, n, t, mode);
   if (need && (!ws || ws_bytes < need)) return fail(TP_ERR_WORKSPACE, "workspace of %zu bytes needed", need);
   if (M == 0) return TP_OK;
+  if (ws && reinterpret_cast<uintptr_t>(ws) % WS_ALIGN)
+    return fail(TP_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
+  if (mode == TP_REDUCE_PARTIALS)
+    TP_TRY(zero_row_counters(static_cast<float*>(ws), M, n, t, static_cast<cudaStream_t>(stream)));
   return run_row(A, M, k / t, n, t, W, bias, residual, 0, out, 0, mode, static_cast<float*>(ws),
                  static_cast<cudaStream_t>(stream));
+}
+
+size_t tp_ffn_backward_workspace_bytes(int64_t M, int64_t h, int64_t f, int t) {
+  if (M <= 0 || h <= 0 || f <= 0 || t < 1) return 0;
+  return ffn_bwd_ws_bytes(M, h, f);
+}
+
+tp_status tp_ffn_backward(const void* X, int64_t M, int64_t h, int64_t f, int t, const tp_shard* W1,
+                          const void* const* b1, const tp_shard* W2, const void* dY, const void* dX_add, void* dX,
+                          float* dW1, float* db1, float* dW2, float* db2, tp_activation act, void* ws,
+                          size_t ws_bytes, tp_stream_t stream) {
+  if (act != TP_ACT_GELU && act != TP_ACT_RELU) return fail(TP_ERR_INVALID_ARG, "unknown activation %d", act);
+  TP_TRY(validate_ffn_bf16_dims(M, h, f, t));
+  // with no rows, X, dY and dX are never touched and may be NULL
+  TP_TRY(check_ptr(X, "X", M > 0));
+  TP_TRY(check_ptr(dY, "dY", M > 0));
+  TP_TRY(check_ptr(dX_add, "dX_add", false));
+  TP_TRY(check_ptr(dX, "dX", M > 0));
+  TP_TRY(check_ptr(dW1, "dW1", true));
+  TP_TRY(check_ptr(dW2, "dW2", true));
+  TP_TRY(check_ptr(db1, "db1", false));
+  TP_TRY(check_ptr(db2, "db2", false));
+  TP_TRY(check_shards(W1, t, f / t, "W1"));
+  TP_TRY(check_shards(W2, t, h, "W2"));
+  TP_TRY(check_bias_array(b1, t, "b1"));
+  if (is_f16(W1) || is_f16(W2)) return fail(TP_ERR_UNSUPPORTED, "the backward pass takes bf16 W1 and W2");
+  if (M > 0 && (dX == X || dX == dY || dX == dX_add)) return fail(TP_ERR_INVALID_ARG, "dX aliases an input");
+  if (M > 0x7FFFFFFF / 2) return fail(TP_ERR_UNSUPPORTED, "too many rows");
+  const size_t need = tp_ffn_backward_workspace_bytes(M, h, f, t);
+  if (need && (!ws || ws_bytes < need))
+    return fail(TP_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws ? ws_bytes : 0);
+  if (ws && (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN))
+    return fail(TP_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M == 0) {
+    // no rows: every weight and bias gradient is zero
+    if (cudaMemsetAsync(dW1, 0, static_cast<size_t>(h) * f * 4, s) != cudaSuccess ||
+        cudaMemsetAsync(dW2, 0, static_cast<size_t>(f) * h * 4, s) != cudaSuccess ||
+        (db1 && cudaMemsetAsync(db1, 0, static_cast<size_t>(f) * 4, s) != cudaSuccess) ||
+        (db2 && cudaMemsetAsync(db2, 0, static_cast<size_t>(h) * 4, s) != cudaSuccess))
+      return fail(TP_ERR_CUDA, "cudaMemsetAsync of the gradients failed");
+    return TP_OK;
+  }
+  return ffn_backward_bf16(X, M, h, f, t, W1, b1, W2, dY, dX_add, dX, dW1, db1, dW2, db2,
+                           act == TP_ACT_GELU ? ACT_GELU : ACT_RELU, ws, s);
 }
 
 size_t tp_attn_workspace_bytes(int B, int S, int h, int heads, int d, int t, tp_reduce_mode mode) {
@@ -650,7 +864,15 @@ tp_status tp_get_device_status(tp_stream_t stream) {
   const uint32_t zero = 0;
   if (cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero)) != cudaSuccess) return fail(TP_ERR_CUDA, "status clear");
   if (v == 0) return TP_OK;
-  if ((v & 0xFF) == DEV_TIMEOUT) return fail(TP_ERR_TIMEOUT, "device wait ran out (site %u)", v >> 8);
+  if ((v & 0xFF) == DEV_TIMEOUT) return fail(TP_ERR_TIMEOUT, "device wait ran out (site %u)", (v >> 8) & 0xFF);
+  if (v & DEV_RANGE_MASK) {
+    std::string where;
+    if (v & DEV_RANGE_COLUMN) where += " column-layer output (act(Z));";
+    if (v & DEV_RANGE_QKV) where += " Q/K/V;";
+    if (v & DEV_RANGE_ATTN_O) where += " attention output O;";
+    if (v & DEV_RANGE_LAYERNORM) where += " LayerNorm output;";
+    return fail(TP_ERR_RANGE, "an fp16 intermediate exceeded 65504 in:%s", where.c_str());
+  }
   return fail(TP_ERR_CUDA, "device status 0x%x", v);
 }
 
@@ -692,6 +914,7 @@ const char* tp_status_string(tp_status s) {
     case TP_ERR_WORKSPACE: return "TP_ERR_WORKSPACE";
     case TP_ERR_CUDA: return "TP_ERR_CUDA";
     case TP_ERR_TIMEOUT: return "TP_ERR_TIMEOUT";
+    case TP_ERR_RANGE: return "TP_ERR_RANGE";
   }
   return "TP_ERR_UNKNOWN";
 }

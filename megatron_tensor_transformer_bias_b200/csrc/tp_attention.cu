@@ -367,6 +367,12 @@ __global__ void __launch_bounds__(THREADS, 2) tp_attention_kernel(const __grid_c
           tmem_ld_32x32b_x32(t_o + c * 32, o);
           tmem_ld_wait();
           if (q < a.S) {
+            if (a.o_f16) {
+              float m = 0.f;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(__uint_as_float(o[i])));
+              note_f16_range(a.status, m * inv, DEV_RANGE_ATTN_O);
+            }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               uint4 w;

@@ -42,13 +42,13 @@ constexpr int EPI_WARPS = 8;                        // two per TMEM sub-partitio
 constexpr int THREADS = 64 + 32 * EPI_WARPS;        // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
 constexpr int STAGING_BYTES = EPI_WARPS * 2 * 2048;   // two 32x32 16-bit buffers per epilogue warp
 constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + 256;
-constexpr uint32_t IDESC_BF16 = idesc_bf16_f32(BM, BN, /*a_mn=*/0, /*b_mn=*/1);
-constexpr uint32_t IDESC_F16 = idesc_f16_f32(BM, BN, /*a_mn=*/0, /*b_mn=*/1);
 
 struct TileCoord {
   int g, m_blk, n_blk;
 };
 
+// Tile order: m fastest, then n, then the group -- so the pairs working at the same time
+// share the group's B tiles through L2.
 __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int tile, int m_tiles, int n_tiles) {
   TileCoord c;
   c.m_blk = tile % m_tiles;
@@ -152,15 +152,17 @@ __device__ __forceinline__ void epilogue_math(const GemmArgs& a, const TileCoord
 // position j ^ ((r >> 1) & 3) of its 64-byte row (no bank conflicts).  Lane 0
 // stores the chunk at (x, y0) and recycles a buffer once the store issued two
 // chunks earlier has read it.
-__device__ __forceinline__ void stage_and_store(const GemmArgs& a, uint8_t* warp_staging, int& count, int lane,
-                                                const float (&v)[32], int x, int y0) {
+__device__ __forceinline__ void stage_and_store(const GemmArgs& a, const CUtensorMap* map, int out_type,
+                                                uint8_t* warp_staging, int& count, int lane, const float (&v)[32],
+                                                int x, int y0) {
   uint8_t* buf = warp_staging + (count & 1) * 2048;
   if (count >= 2) {
     if (lane == 0) bulk_wait_group_read<1>();
     __syncwarp();
   }
   uint32_t pk[16];
-  if (a.out_type == OUT_F16) {
+  if (out_type == OUT_F16) {
+    note_f16_range(a.status, absmax32(v), DEV_RANGE_COLUMN);
 #pragma unroll
     for (int i = 0; i < 16; ++i) pk[i] = pack_f16x2(v[2 * i], v[2 * i + 1]);
   } else {
@@ -175,10 +177,176 @@ __device__ __forceinline__ void stage_and_store(const GemmArgs& a, uint8_t* warp
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0 && y0 < a.M) {
-    tma_store_2d(&a.tmOut, buf, x, y0);
+    tma_store_2d(map, buf, x, y0);
     bulk_commit_group();
   }
   ++count;
+}
+
+__device__ __forceinline__ void load_f16x32(const void* p, float (&v)[32]) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 u = __ldg(q + i);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[j]));
+      v[i * 8 + j * 2] = f.x;
+      v[i * 8 + j * 2 + 1] = f.y;
+    }
+  }
+}
+
+// One 32-column chunk of an epilogue whose 16-bit output leaves through TMA stores.
+// `x` is the chunk's first output column, `y0` the first row of the warp's 32 rows.
+__device__ __forceinline__ void epilogue_tma_chunk(const GemmArgs& a, const TileCoord& tc, int row, int n,
+                                                   float (&v)[32], uint8_t* warp_staging, int& count, int lane,
+                                                   int x, int y0) {
+  if (a.epi == EPI_ACT_GRAD) {
+    // the backward's recomputation of the column layer: act(z) and act'(z), z = acc + b
+    if (a.bias_g[tc.g]) {
+      float b[32];
+      load_bf16x32(static_cast<const uint16_t*>(a.bias_g[tc.g]) + n, b);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] += b[j];
+    }
+    float gr[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = act_and_grad(v[j], a.act, gr[j]);
+    stage_and_store(a, &a.tmOut, a.out_type, warp_staging, count, lane, v, x, y0);
+    stage_and_store(a, &a.tmOut2, OUT_F16, warp_staging, count, lane, gr, x, y0);
+    return;
+  }
+  if (a.epi == EPI_MUL_GRAD) {
+    // dZ = dA * act'(Z): the factor sits at the output's own position
+    if (row < a.M) {
+      float gm[32];
+      load_f16x32(static_cast<const uint16_t*>(a.grad_mul) + static_cast<int64_t>(row) * a.ld_grad + x, gm);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] *= gm[j];
+    }
+    stage_and_store(a, &a.tmOut, a.out_type, warp_staging, count, lane, v, x, y0);
+    return;
+  }
+  epilogue_math(a, tc, row, n, v);
+  stage_and_store(a, &a.tmOut, a.out_type, warp_staging, count, lane, v, x, y0);
+}
+
+__device__ __forceinline__ void load_f32x32_cg(const float* p, float (&v)[32]) {
+  const float4* q = reinterpret_cast<const float4*>(p);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 u = __ldcg(q + i);
+    v[i * 4] = u.x; v[i * 4 + 1] = u.y; v[i * 4 + 2] = u.z; v[i * 4 + 3] = u.w;
+  }
+}
+
+// Step 3 inside the row GEMM (partials mode, a.red_out set).  Tiles run in the order
+// m, n, group, so in every CTA pair's sequence all tiles of groups 0..G-2 come before any
+// tile of group G-1.  A warp of a group g < G-1 tile stores its 32-row x 128-column region
+// of the fp32 partial P_g and counts it on the region's arrival counter.  The warp of the
+// group G-1 tile that covers the same region waits (bounded) until the G-1 earlier
+// partials are counted -- they were stored before their pairs started any group G-1
+// tile, so the wait always ends -- and then sums P_0 .. P_{G-2} from memory and its own
+// P_{G-1} straight from the accumulator, in the order 0..G-1, adds bias and residual and
+// writes the output.  P_{G-1} is never stored.  The sums are those of a separate pass
+// over the stored partials: same order, same bits.
+
+// Arrival counter of the region (32 rows from row0, the 128 columns of col_region).
+__device__ __forceinline__ int region_counter(const GemmArgs& a, int row0, int col_region) {
+  return (row0 / 32) * ((a.N + 127) / 128) + col_region;
+}
+
+// Publish this warp's stores of its region of a partial: each lane's stores are fenced
+// before lane 0's atomic.
+__device__ __forceinline__ void partial_signal(const GemmArgs& a, int ctr, int lane) {
+  __threadfence();
+  __syncwarp();
+  if (lane == 0) atomicAdd(&a.counters[ctr], 1u);
+}
+
+// Wait until the region's G-1 earlier partials are counted; fenced so that the warp's
+// later loads see them.  false: the wait ran out (recorded in the status word).
+__device__ __forceinline__ bool partial_wait(const GemmArgs& a, int ctr, int lane) {
+  int ok = 1;
+  if (lane == 0) {
+    const volatile uint32_t* c = a.counters + ctr;
+    const uint32_t want = static_cast<uint32_t>(a.G - 1);
+    if (*c < want) {
+      const uint64_t t0 = globaltimer_ns();
+      while (*c < want) {
+        if (globaltimer_ns() - t0 > a.wait_limit_ns) {
+          record_status(a.status, DEV_TIMEOUT, WAIT_SITE_EPILOGUE);
+          ok = 0;
+          break;
+        }
+      }
+    }
+    __threadfence();
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  __threadfence();
+  return ok != 0;
+}
+
+// One 32-column chunk of a group G-1 tile: out = ((P_0 + P_1) + ...) + P_{G-1} + bias + resid,
+// taken 16 columns at a time (the result replaces v) to keep the registers in check.  The
+// partials were written earlier in this launch: they are read with plain (L1-allocating)
+// loads, never through the read-only path, and no line of them was in this SM's L1 before.
+__device__ __forceinline__ void reduce_chunk(const GemmArgs& a, int row, int n, float (&v)[32], bool ok,
+                                             uint8_t* warp_staging, int& count, int lane) {
+  if (row < a.M && ok) {
+    const float* p = static_cast<const float*>(a.out) + static_cast<int64_t>(row) * a.ld_out + n;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      float acc[16];
+      if (a.G > 1) {
+        const float4* q0 = reinterpret_cast<const float4*>(p + half * 16);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 u = q0[i];
+          acc[i * 4] = u.x; acc[i * 4 + 1] = u.y; acc[i * 4 + 2] = u.z; acc[i * 4 + 3] = u.w;
+        }
+        for (int g = 1; g < a.G - 1; ++g) {
+          const float4* q = reinterpret_cast<const float4*>(p + static_cast<int64_t>(g) * a.out_group_stride + half * 16);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float4 u = q[i];
+            acc[i * 4] += u.x; acc[i * 4 + 1] += u.y; acc[i * 4 + 2] += u.z; acc[i * 4 + 3] += u.w;
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) acc[j] += v[half * 16 + j];
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) acc[j] = v[half * 16 + j];
+      }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[half * 16 + j] = acc[j];
+    }
+    if (a.bias) {
+      float b[32];
+      load_bf16x32(static_cast<const uint16_t*>(a.bias) + n, b);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] += b[j];
+    }
+    if (a.resid) {
+      float r[32];
+      if (a.resid_fp32)
+        load_f32x32(static_cast<const float*>(a.resid) + static_cast<int64_t>(row) * a.ld_resid + n, r);
+      else
+        load_bf16x32(static_cast<const uint16_t*>(a.resid) + static_cast<int64_t>(row) * a.ld_resid + n, r);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] += r[j];
+    }
+  }
+  if (a.red_out_f32) {
+    if (row < a.M) store_f32x32(static_cast<float*>(a.red_out) + static_cast<int64_t>(row) * a.N + n, v);
+  } else {
+    stage_and_store(a, &a.tmOut, OUT_BF16, warp_staging, count, lane, v, n, row - lane);
+  }
 }
 
 // One 32-column chunk of one accumulator row: apply the epilogue and store.
@@ -194,6 +362,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, const TileCoor
       }
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] = act_apply(v[j], a.act);
+      if (a.out_type == OUT_F16) note_f16_range(a.status, absmax32(v), DEV_RANGE_COLUMN);
       store_x32(a.out, static_cast<int64_t>(row) * a.ld_out + static_cast<int64_t>(tc.g) * a.out_col_per_group + n,
                 a.out_type, v);
       break;
@@ -240,6 +409,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, const TileCoor
       void* base = part == 0 ? a.q : (part == 1 ? a.k : a.v);
       uint16_t* o = static_cast<uint16_t*>(base) +
                     ((static_cast<int64_t>(b) * a.H + head) * a.S + s) * a.d + dd;
+      note_f16_range(a.status, absmax32(v), DEV_RANGE_QKV);
       store_f16x32(o, v);
       break;
     }
@@ -271,7 +441,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
   const int m_tiles = (a.M + BM - 1) / BM;
   const int n_tiles = (a.N + BN - 1) / BN;
   const int num_tiles = m_tiles * n_tiles * (a.concat ? 1 : a.G);
-  const int kb_per_group = a.Kg / BK;
+  const int kb_per_group = (a.Kg + BK - 1) / BK;   // a ragged last K step reads zero fill
   const int k_iters = a.concat ? kb_per_group * a.G : kb_per_group;
 
   if (threadIdx.x == 0) {
@@ -323,12 +493,21 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
           const int g = a.concat ? it / kb_per_group : tc.g;
           const int kb = a.concat ? it - g * kb_per_group : it;
           mbar_arrive_expect_tx(&full_bar[stage], STAGE_BYTES);
-          tma_load_2d_hint(sA + stage * A_STAGE_BYTES, &a.tmA, &full_bar[stage], g * a.a_k_per_group + kb * BK, m0,
-                           pol_a);
+          uint8_t* a_dst = sA + stage * A_STAGE_BYTES;
+          const int ka = g * a.a_k_per_group + kb * BK;
+          if (!a.a_mn) {
+            tma_load_2d_hint(a_dst, &a.tmA, &full_bar[stage], ka, m0, pol_a);
+          } else {  // two 64-wide M blocks of 64 K rows
+            tma_load_3d_hint(a_dst, &a.tmA, &full_bar[stage], 0, ka, (g * a.a_m_per_group + m0) / 64, pol_a);
+          }
           uint8_t* b_dst = sB + stage * B_STAGE_BYTES;
-#pragma unroll
-          for (int j = 0; j < BN / 64; ++j)
-            tma_load_2d_hint(b_dst + j * B_BLOCK_BYTES, &a.tmB[g], &full_bar[stage], n0 + j * 64, kb * BK, pol_b);
+          if (!a.b_kmajor) {  // four 64-wide N blocks of 64 K rows, two per load
+            tma_load_3d_hint(b_dst, &a.tmB[g], &full_bar[stage], 0, kb * BK, n0 / 64, pol_b);
+            tma_load_3d_hint(b_dst + 2 * B_BLOCK_BYTES, &a.tmB[g], &full_bar[stage], 0, kb * BK, n0 / 64 + 2, pol_b);
+          } else {  // two 128-row N blocks of 64 K each
+            tma_load_2d_hint(b_dst, &a.tmB[g], &full_bar[stage], kb * BK, n0, pol_b);
+            tma_load_2d_hint(b_dst + BN / 2 * 128, &a.tmB[g], &full_bar[stage], kb * BK, n0 + BN / 2, pol_b);
+          }
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -350,7 +529,8 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      const uint32_t idesc = a.ab_f16 ? IDESC_F16 : IDESC_BF16;
+      const uint32_t idesc = a.ab_f16 ? idesc_f16_f32(BM, BN, a.a_mn, !a.b_kmajor)
+                                      : idesc_bf16_f32(BM, BN, a.a_mn, !a.b_kmajor);
       const uint32_t sA_addr = smem_u32(sA);
       const uint32_t sB_addr = smem_u32(sB);
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
@@ -369,10 +549,12 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
           const uint32_t b_base = sB_addr + stage * B_STAGE_BYTES;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
-            // A: K-major, advance 16 elements (32 bytes) inside the swizzle atom.
-            const uint64_t adesc = smem_desc_sw128(a_base + k * 32, 16, 1024);
-            // B: N-major, advance 16 K-rows (2048 bytes); 64-column blocks 8 KB apart.
-            const uint64_t bdesc = smem_desc_sw128(b_base + k * 16 * 128, B_BLOCK_BYTES, 1024);
+            // K-major operand: advance 16 elements (32 bytes) inside the swizzle atom;
+            // MN-major operand: advance 16 K-rows (2048 bytes), 64-wide MN blocks 8 KB apart.
+            const uint64_t adesc = a.a_mn ? smem_desc_sw128(a_base + k * 16 * 128, B_BLOCK_BYTES, 1024)
+                                          : smem_desc_sw128(a_base + k * 32, 16, 1024);
+            const uint64_t bdesc = a.b_kmajor ? smem_desc_sw128(b_base + k * 32, 16, 1024)
+                                              : smem_desc_sw128(b_base + k * 16 * 128, B_BLOCK_BYTES, 1024);
             mma_bf16_ss(d_tmem, adesc, bdesc, idesc, (it > 0 || k > 0) ? 1u : 0u);
           }
           mma_commit(&empty_bar[stage]);  // frees the smem stage once these MMAs finish
@@ -393,7 +575,8 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
     const int col_half = (warp - 2) / 4;    // columns [col_half*BN/2, +BN/2) of each tile
     int acc = 0;
     uint32_t acc_phase = 0;
-    const bool tma_out = a.tma_store && (a.epi == EPI_ACT || a.epi == EPI_BIAS_RESID);
+    const bool tma_out = a.tma_store && (a.epi == EPI_ACT || a.epi == EPI_BIAS_RESID || a.epi == EPI_ACT_GRAD ||
+                                         a.epi == EPI_MUL_GRAD);
     uint8_t* warp_staging = staging + (warp - 2) * 4096;
     int store_count = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -416,6 +599,16 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
       const int c_begin = col_half * (BN / 64);
       int c_end = (col_half + 1) * (BN / 64);
       if (n0 + c_end * 32 > a.N) c_end = (a.N - n0) / 32;
+      // partials mode with the reduction here: this warp's region and its role in it
+      const int row0 = tc.m_blk * BM + sub * 32;
+      const bool in_region = a.red_out && row0 < a.M && c_begin < c_end;
+      const int ctr = in_region ? region_counter(a, row0, n0 / 128 + col_half) : 0;
+      const bool red_tile = a.red_out && tc.g == a.G - 1;
+      bool red_ok = true;
+      if (red_tile && in_region) {
+        red_ok = partial_wait(a, ctr, lane);
+        if (!red_ok) *abort_flag = 1;
+      }
       if (c_begin < c_end) {
         uint32_t r[2][32];
         tmem_ld_32x32b_x32(t_row + c_begin * 32, r[0]);
@@ -428,10 +621,11 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
           float v[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[cur][j]);
-          if (tma_out) {
-            epilogue_math(a, tc, row, n0 + c * 32, v);
-            const int x = (a.epi == EPI_ACT ? tc.g * static_cast<int>(a.out_col_per_group) : 0) + n0 + c * 32;
-            stage_and_store(a, warp_staging, store_count, lane, v, x, row - lane);
+          if (red_tile) {
+            reduce_chunk(a, row, n0 + c * 32, v, red_ok, warp_staging, store_count, lane);
+          } else if (tma_out) {
+            const int x = (a.epi == EPI_BIAS_RESID ? 0 : tc.g * static_cast<int>(a.out_col_per_group)) + n0 + c * 32;
+            epilogue_tma_chunk(a, tc, row, n0 + c * 32, v, warp_staging, store_count, lane, x, row - lane);
           } else if (row < a.M) {
             epilogue_chunk(a, tc, row, n0 + c * 32, v);
           }
@@ -442,6 +636,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
       if (++acc == NUM_ACC) { acc = 0; acc_phase ^= 1u; }
+      if (in_region && !red_tile) partial_signal(a, ctr, lane);
     }
     if (lane == 0) bulk_wait_group_all();  // our output stores are complete before exit
   }
@@ -471,8 +666,6 @@ constexpr int P_A_BYTES = BM * BK * 2;              // 16 KB per CTA
 constexpr int P_B_BYTES = (BN / 2) * BK * 2;        // 16 KB per CTA
 constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
 constexpr int P_SMEM_BYTES = 1024 + P_STAGES * P_STAGE_BYTES + STAGING_BYTES + 256;
-constexpr uint32_t P_IDESC_BF16 = idesc_bf16_f32(P_ROWS, BN, 0, 1);
-constexpr uint32_t P_IDESC_F16 = idesc_f16_f32(P_ROWS, BN, 0, 1);
 
 __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_constant__ GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -500,7 +693,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
   const int m_tiles = (a.M + P_ROWS - 1) / P_ROWS;
   const int n_tiles = (a.N + BN - 1) / BN;
   const int num_tiles = m_tiles * n_tiles * (a.concat ? 1 : a.G);
-  const int kb_per_group = a.Kg / BK;
+  const int kb_per_group = (a.Kg + BK - 1) / BK;   // a ragged last K step reads zero fill
   const int k_iters = a.concat ? kb_per_group * a.G : kb_per_group;
 
   if (threadIdx.x == 0) {
@@ -559,10 +752,19 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
           const int kb = a.concat ? kidx - g * kb_per_group : kidx;
           const uint32_t fb = full0_leader + static_cast<uint32_t>(stage) * 8u;
           if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * P_STAGE_BYTES);
-          tma_load_2d_pair(sA + stage * P_A_BYTES, &a.tmA, fb, g * a.a_k_per_group + kb * BK, m0, pol_a);
+          uint8_t* a_dst = sA + stage * P_A_BYTES;
+          const int ka = g * a.a_k_per_group + kb * BK;
+          if (!a.a_mn) {
+            tma_load_2d_pair(a_dst, &a.tmA, fb, ka, m0, pol_a);
+          } else {  // two 64-wide M blocks of 64 K rows, one load
+            tma_load_3d_pair(a_dst, &a.tmA, fb, 0, ka, (g * a.a_m_per_group + m0) / 64, pol_a);
+          }
           uint8_t* b_dst = sB + stage * P_B_BYTES;
-          tma_load_2d_pair(b_dst, &a.tmB[g], fb, n0, kb * BK, pol_b);
-          tma_load_2d_pair(b_dst + B_BLOCK_BYTES, &a.tmB[g], fb, n0 + 64, kb * BK, pol_b);
+          if (!a.b_kmajor) {  // this CTA's two 64-wide N blocks of 64 K rows, one load
+            tma_load_3d_pair(b_dst, &a.tmB[g], fb, 0, kb * BK, n0 / 64, pol_b);
+          } else {  // this CTA's 128 N rows, 64 K each
+            tma_load_2d_pair(b_dst, &a.tmB[g], fb, kb * BK, n0, pol_b);
+          }
           ++issued;
           if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -580,7 +782,8 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader only)
     if (lane == 0 && leader) {
-      const uint32_t idesc = a.ab_f16 ? P_IDESC_F16 : P_IDESC_BF16;
+      const uint32_t idesc = a.ab_f16 ? idesc_f16_f32(P_ROWS, BN, a.a_mn, !a.b_kmajor)
+                                      : idesc_bf16_f32(P_ROWS, BN, a.a_mn, !a.b_kmajor);
       const uint32_t sA_addr = smem_u32(sA);
       const uint32_t sB_addr = smem_u32(sB);
       int stage = 0;
@@ -604,8 +807,10 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
           const uint32_t b_base = sB_addr + stage * P_B_BYTES;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
-            const uint64_t adesc = smem_desc_sw128(a_base + k * 32, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(b_base + k * 16 * 128, B_BLOCK_BYTES, 1024);
+            const uint64_t adesc = a.a_mn ? smem_desc_sw128(a_base + k * 16 * 128, B_BLOCK_BYTES, 1024)
+                                          : smem_desc_sw128(a_base + k * 32, 16, 1024);
+            const uint64_t bdesc = a.b_kmajor ? smem_desc_sw128(b_base + k * 32, 16, 1024)
+                                              : smem_desc_sw128(b_base + k * 16 * 128, B_BLOCK_BYTES, 1024);
             mma_pair_ss(d_tmem, adesc, bdesc, idesc, (it > 0 || k > 0) ? 1u : 0u);
           }
           mma_commit_pair_mask(&empty_bar[stage], 0x3);  // frees this stage in both CTAs
@@ -626,7 +831,8 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
     const uint32_t acc_empty0_leader = mapa_shared(smem_u32(&acc_empty[0]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
-    const bool tma_out = a.tma_store && (a.epi == EPI_ACT || a.epi == EPI_BIAS_RESID);
+    const bool tma_out = a.tma_store && (a.epi == EPI_ACT || a.epi == EPI_BIAS_RESID || a.epi == EPI_ACT_GRAD ||
+                                         a.epi == EPI_MUL_GRAD);
     uint8_t* warp_staging = staging + (warp - 2) * 4096;
     int store_count = 0;
     for (int tile = cid; tile < num_tiles; tile += nclusters) {
@@ -648,6 +854,16 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
       const int c_begin = col_half * (BN / 64);
       int c_end = (col_half + 1) * (BN / 64);
       if (n0 + c_end * 32 > a.N) c_end = (a.N - n0) / 32;
+      // partials mode with the reduction here: this warp's region and its role in it
+      const int row0 = tc.m_blk * P_ROWS + static_cast<int>(rank) * BM + sub * 32;
+      const bool in_region = a.red_out && row0 < a.M && c_begin < c_end;
+      const int ctr = in_region ? region_counter(a, row0, n0 / 128 + col_half) : 0;
+      const bool red_tile = a.red_out && tc.g == a.G - 1;
+      bool red_ok = true;
+      if (red_tile && in_region) {
+        red_ok = partial_wait(a, ctr, lane);
+        if (!red_ok) *abort_flag = 1;
+      }
       if (c_begin < c_end) {
         uint32_t r[2][32];
         tmem_ld_32x32b_x32(t_row + c_begin * 32, r[0]);
@@ -660,10 +876,11 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
           float v[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[cur][j]);
-          if (tma_out) {
-            epilogue_math(a, tc, row, n0 + c * 32, v);
-            const int x = (a.epi == EPI_ACT ? tc.g * static_cast<int>(a.out_col_per_group) : 0) + n0 + c * 32;
-            stage_and_store(a, warp_staging, store_count, lane, v, x, row - lane);
+          if (red_tile) {
+            reduce_chunk(a, row, n0 + c * 32, v, red_ok, warp_staging, store_count, lane);
+          } else if (tma_out) {
+            const int x = (a.epi == EPI_BIAS_RESID ? 0 : tc.g * static_cast<int>(a.out_col_per_group)) + n0 + c * 32;
+            epilogue_tma_chunk(a, tc, row, n0 + c * 32, v, warp_staging, store_count, lane, x, row - lane);
           } else if (row < a.M) {
             epilogue_chunk(a, tc, row, n0 + c * 32, v);
           }
@@ -674,6 +891,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty0_leader + static_cast<uint32_t>(acc) * 8u);
       if (++acc == NUM_ACC) { acc = 0; acc_phase ^= 1u; }
+      if (in_region && !red_tile) partial_signal(a, ctr, lane);
     }
     if (lane == 0) bulk_wait_group_all();  // our output stores are complete before exit
   }

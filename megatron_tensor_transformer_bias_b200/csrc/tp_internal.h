@@ -10,8 +10,19 @@
 
 namespace tpb {
 
-// Device status word codes (the low byte; the next byte says where a wait gave up).
+// Device status word.  Low byte: the code of the first failure (DEV_TIMEOUT), next
+// byte: where that wait gave up.  Bits 16..19: a value that an epilogue was about to
+// store in fp16 exceeded the largest fp16 number (65504), one bit per producing site;
+// these are OR-ed in and do not stop the kernel.
 enum : uint32_t { DEV_OK = 0, DEV_TIMEOUT = 5 };
+enum : uint32_t {
+  DEV_RANGE_COLUMN = 1u << 16,   // column layer output (act(Z) or a column linear), fp16
+  DEV_RANGE_QKV = 1u << 17,      // Q, K, V of the attention projection (always fp16)
+  DEV_RANGE_ATTN_O = 1u << 18,   // attention output O, fp16
+  DEV_RANGE_LAYERNORM = 1u << 19,  // LayerNorm output, fp16
+  DEV_RANGE_MASK = 0xFu << 16
+};
+constexpr float FP16_MAX = 65504.0f;
 enum : uint32_t {
   WAIT_SITE_PRODUCER = 1, WAIT_SITE_MMA_FULL = 2, WAIT_SITE_MMA_ACC = 3,
   WAIT_SITE_EPILOGUE = 4, WAIT_SITE_SELFTEST = 5, WAIT_SITE_ATTN = 6
@@ -27,6 +38,8 @@ enum GemmEpilogue : int {
   EPI_PARTIAL_F32 = 1, // P[g][m, n] = acc as fp32                              (row layer, partials)
   EPI_BIAS_RESID = 2,  // out[m, n] = acc + bias[n] + resid[m, n]              (row layer, fused reduce)
   EPI_QKV = 3,         // scatter acc (+ bias_g) to Q/K/V [B, H, S, d] fp16     (QKV column layer)
+  EPI_ACT_GRAD = 4,    // z = acc + bias_g: out = act(z) (16-bit), out2 = act'(z) (fp16)  (backward recompute)
+  EPI_MUL_GRAD = 5,    // out[:, g*ncol + n] = acc * grad_mul[:, g*ncol + n] (fp16 factor)  (backward dZ)
 };
 
 // Element type of an epilogue output.
@@ -35,12 +48,20 @@ enum OutType : int { OUT_BF16 = 0, OUT_F32 = 1, OUT_F16 = 2 };
 enum Activation : int { ACT_NONE = 0, ACT_GELU = 1, ACT_RELU = 2 };
 
 struct __align__(64) GemmArgs {
-  CUtensorMap tmOut;                    // 16-bit output of EPI_ACT / EPI_BIAS_RESID, box {32, 32}, 64B swizzle
-  CUtensorMap tmA;                      // A [M, Ktot] bf16 K-major, box {64, 128}, 128B swizzle
-  CUtensorMap tmB[TP_MAX_SHARDS];       // B_g [Kg, N] bf16 N-major, box {64, 64}, 128B swizzle
+  CUtensorMap tmOut;                    // 16-bit output of the TMA-store epilogues, box {32, 32}, 64B swizzle
+  CUtensorMap tmOut2;                   // EPI_ACT_GRAD: act'(z) output (fp16), same box
+  // A [M, Ktot] K-major: box {64 K, 128 M}; or (a_mn) the matrix [Ktot, M] with M
+  // contiguous: a make_tmap_mn map (box {64 M, 64 K, 2 blocks}).  128B swizzle.
+  CUtensorMap tmA;
+  // B_g [Kg, N] N-major: a make_tmap_mn map (box {64 N, 64 K, 2 blocks}); or (b_kmajor) the
+  // matrix [N, Kg] with K contiguous: box {64 K, 128 N}.  128B swizzle.
+  CUtensorMap tmB[TP_MAX_SHARDS];
   int M, N, Kg, G;
   int concat;                           // 1: one tile sums all G K-slices in order g = 0..G-1
   int a_k_per_group;                    // column offset of group g's K-slice in A (elements)
+  int a_m_per_group;                    // a_mn: M offset of group g's rows in A's map (elements)
+  int a_mn;                             // A is M-major (the transpose of a row-major [K, M] matrix)
+  int b_kmajor;                         // B is K-major (the transpose of a row-major [N, K] matrix)
   int epi, act;
   int ab_f16;                           // A and B operands are fp16 (else bf16)
   void* out;
@@ -54,12 +75,25 @@ struct __align__(64) GemmArgs {
   const void* resid;                    // [M, N] or null
   int64_t ld_resid;
   int resid_fp32;
+  // EPI_MUL_GRAD: fp16 factor [M, ld_grad] read at the output's column
+  const void* grad_mul;
+  int64_t ld_grad;
   // EPI_QKV scatter: column c of group g -> part c / (Hg*d), head g*Hg + (c % (Hg*d)) / d
   void* q; void* k; void* v;
   int S, H, Hg, d;
+  // EPI_PARTIAL_F32 with the reduction in the epilogue (red_out != null): one arrival
+  // counter per 32-row x 128-column region of the output, zero on entry.  The epilogue
+  // warp whose arrival completes a region's G partials sums them in order g = 0..G-1,
+  // adds bias and resid and writes red_out [M, N] (fp32 if red_out_f32, else bf16).
+  uint32_t* counters;
+  void* red_out;
+  int red_out_f32;
   uint32_t* status;
   uint64_t wait_limit_ns;
 };
+
+// Arrival counters of the in-epilogue reduction: one per 32-row x 128-column region.
+inline size_t partial_counter_count(int64_t M, int64_t N) { return static_cast<size_t>((M + 31) / 32) * ((N + 127) / 128); }
 
 struct AttnArgs {
   CUtensorMap tmQ;   // Q [B*H][S][d] fp16, box {64, 128, 1}, 128B swizzle
@@ -83,6 +117,11 @@ uint64_t wait_limit_ns();
 // 2-byte element tensor maps (bf16 or fp16), 128-byte swizzle, zero fill out of bounds.
 tp_status make_tmap_2d(CUtensorMap* map, const void* base, int f16, uint64_t inner, uint64_t outer,
                        uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+// Map of an MN-major operand ([k_rows, mn_cols] row-major, MN contiguous, mn_cols % 64 == 0):
+// 3-D view (64, k_rows, mn_cols / 64), box {64, 64, 2}: one load brings two 64-wide MN
+// blocks of 64 K rows, 8 KB apart in shared memory.  128-byte swizzle, zero fill.
+tp_status make_tmap_mn(CUtensorMap* map, const void* base, int f16, uint64_t mn_cols, uint64_t k_rows,
+                       uint64_t row_stride_bytes);
 // Output map of the epilogue stores: box {32, 32} of a 2-byte type, 64-byte swizzle.
 tp_status make_tmap_out(CUtensorMap* map, void* base, int f16, uint64_t cols, uint64_t rows,
                         uint64_t row_stride_bytes);
@@ -100,14 +139,20 @@ tp_status launch_ffn_fp32(const float* X, int64_t M, int64_t h, int64_t f, int t
                           const void* const* b1, const tp_shard* W2, const float* b2, const float* resid,
                           float* out, int act, float* Z, float* P, cudaStream_t stream);
 tp_status launch_selftest_wait(uint64_t limit_ns, cudaStream_t stream);
+// out[c] = sum_r x[r, c] (bf16 x [M, ld], fp32 out [n]) in a fixed order, through `part`
+// (colsum_workspace_bytes(M, n) bytes of fp32 scratch).
+size_t colsum_workspace_bytes(int64_t M, int64_t n);
+tp_status launch_colsum(const void* x, int64_t M, int64_t n, int64_t ld, float* part, float* out,
+                        cudaStream_t stream);
 tp_status launch_act(const float* x, float* y, int64_t n, int act, cudaStream_t stream);
 
-// Launch `kern` on `stream` with programmatic dependent launch (the kernel waits for
-// its predecessor with griddepcontrol.wait before touching global memory) and an
 // Record `msg` as the calling thread's tp_last_error() and return `s`.
 tp_status set_error(tp_status s, const char* msg);
-// optional cluster size.  TPB_PDL=0 turns the attribute off.
+// Whether launches carry the programmatic-dependent-launch attribute (TPB_PDL=0: no).
 bool pdl_enabled();
+// Launch `kern` on `stream` with programmatic dependent launch (the kernel waits for
+// its predecessor with griddepcontrol.wait before touching global memory) and an
+// optional cluster size.
 template <typename... KArgs, typename... Args>
 tp_status launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, int cluster_x,
                     Args&&... args) {

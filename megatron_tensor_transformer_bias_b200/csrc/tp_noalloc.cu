@@ -8,7 +8,7 @@
 // and outputs; the intermediate act(Z) goes to `g_ffn_scratch` below.
 //
 // Limits and sharing:
-//  * The scratch holds TP_NOALLOC_SCRATCH_BYTES = 16 MiB, i.e. M * f <= 8,388,608
+//  * The scratch holds kScratchBytes = 16 MiB, i.e. M * f <= 8,388,608
 //    bf16 elements; larger calls are rejected with TP_ERR_UNSUPPORTED.
 //  * Every GPU that loads the library holds the array until the process exits.
 //  * Every call on a device shares the one array, which keeps the last call's
@@ -17,7 +17,9 @@
 //    GPU (for example on two streams) race on the array and give wrong results.
 //  * The first call on each device looks up the array's device address
 //    (cudaGetSymbolAddress, with that device current); make that first call
-//    before any stream capture.
+//    before any stream capture.  Later calls look it up again unless their
+//    stream is capturing, so a device reset (which reloads the module and may
+//    move the array) does not leave a stale address behind.
 #include <atomic>
 #include <cstdio>
 
@@ -34,13 +36,19 @@ static __device__ __align__(256) unsigned char g_ffn_scratch[kScratchBytes];
 constexpr int kMaxDevices = 64;
 std::atomic<void*> g_scratch_addr[kMaxDevices];
 
-// Device address of g_ffn_scratch on the current device (looked up once per device).
-tp_status scratch_address(void** out) {
+// Device address of g_ffn_scratch on the current device: looked up on every call whose
+// stream is not being captured, reused from the last lookup while it is.
+tp_status scratch_address(cudaStream_t stream, void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return tpb::set_error(TP_ERR_CUDA, "cudaGetDevice failed");
   if (dev < 0 || dev >= kMaxDevices) return tpb::set_error(TP_ERR_UNSUPPORTED, "device index above 63");
-  void* p = g_scratch_addr[dev].load();
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess)
+    return tpb::set_error(TP_ERR_CUDA, "cudaStreamIsCapturing failed");
+  void* p = cap == cudaStreamCaptureStatusNone ? nullptr : g_scratch_addr[dev].load();
   if (!p) {
+    if (cap != cudaStreamCaptureStatusNone)
+      return tpb::set_error(TP_ERR_INVALID_ARG, "first no-allocation call on this device is being captured");
     const cudaError_t e = cudaGetSymbolAddress(&p, g_ffn_scratch);
     if (e != cudaSuccess || !p) {
       char msg[160];
@@ -74,7 +82,7 @@ extern "C" tp_status tp_ffn_forward_noalloc(const void* X, int64_t M, int64_t h,
   if (out && (out == X || out == residual)) return tpb::set_error(TP_ERR_INVALID_ARG, "out aliases an input");
   if (M == 0) return TP_OK;
   void* scratch = nullptr;
-  const tp_status s = scratch_address(&scratch);
+  const tp_status s = scratch_address(static_cast<cudaStream_t>(stream), &scratch);
   if (s != TP_OK) return s;
   // step 1: act(Z) = GeLU(X W1_i + b1_i) for every shard, into the static scratch [M, f]
   const tp_status c = tp_column_linear_forward(X, M, h, f, t, W1, b1, TP_ACT_GELU, scratch, stream);

@@ -80,9 +80,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Record the first failure only; the host reads and clears the word.
+// Record the first failure only (low 16 bits); the host reads and clears the word.
+// Range bits already OR-ed into the high half are kept.
 __device__ __forceinline__ void record_status(uint32_t* status, uint32_t code, uint32_t site) {
-  if (status) atomicCAS(status, 0u, code | (site << 8));
+  if (!status) return;
+  uint32_t old = *reinterpret_cast<volatile uint32_t*>(status);
+  while ((old & 0xFFFFu) == 0) {
+    const uint32_t prev = atomicCAS(status, old, old | code | (site << 8));
+    if (prev == old) break;
+    old = prev;
+  }
+}
+
+// An fp16 store is about to take a value of magnitude `amax`: above 65504 it would
+// become +-inf, so the producing site's bit goes into the status word (the store
+// itself still happens; tp_get_device_status then reports TP_ERR_RANGE).
+__device__ __forceinline__ void note_f16_range(uint32_t* status, float amax, uint32_t site_bit) {
+  if (amax > FP16_MAX && status) atomicOr(status, site_bit);
+}
+
+// Largest |v[i]| of a 32-value chunk (NaN inputs are ignored by fmaxf).
+__device__ __forceinline__ float absmax32(const float (&v)[32]) {
+  float m0 = 0.f, m1 = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    m0 = fmaxf(m0, fabsf(v[i]));
+    m1 = fmaxf(m1, fabsf(v[i + 1]));
+  }
+  return fmaxf(m0, m1);
 }
 
 // Wait until the phase with parity `parity` of `bar` has completed, for at most
@@ -266,6 +291,27 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const void* tma
       : "memory");
 }
 
+// 3-D tiled load (a make_tmap_mn map: x = 0, y = K row, z = 64-wide MN block) into this
+// CTA's shared memory, bytes counted on the pair leader's barrier; no multicast.
+__device__ __forceinline__ void tma_load_3d_pair(void* smem_dst, const void* tmap, uint32_t bar_cluster, int32_t x,
+                                                 int32_t y, int32_t z, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
+      "[%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster), "r"(x), "r"(y), "r"(z), "l"(policy)
+      : "memory");
+}
+
+// 3-D tiled load into this CTA's shared memory, completion on its own barrier.
+__device__ __forceinline__ void tma_load_3d_hint(void* smem_dst, const void* tmap, uint64_t* bar, int32_t x,
+                                                 int32_t y, int32_t z, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, "
+      "%4, %5}], [%2], %6;" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* smem_result, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_result)),
                "r"(ncols)
@@ -355,6 +401,39 @@ __device__ __forceinline__ float gelu_exact(float x) {
   p = fmaf(p, t, -1.26551223f);
   const float half_erfc = 0.5f * t * __expf(fmaf(-z, z, p));
   return x * (x >= 0.0f ? 1.0f - half_erfc : half_erfc);
+}
+
+// GeLU and its derivative together: GeLU'(x) = Phi(x) + x phi(x), phi(x) = exp(-x^2/2) / sqrt(2 pi),
+// with Phi from the same erfc formula as gelu_exact (so GeLU here is bit-identical to it).
+__device__ __forceinline__ float gelu_and_grad(float x, float& grad) {
+  const float z = fabsf(x) * 0.70710678118654752f;
+  const float t = __fdividef(1.0f, fmaf(0.5f, z, 1.0f));
+  float p = 0.17087277f;
+  p = fmaf(p, t, -0.82215223f);
+  p = fmaf(p, t, 1.48851587f);
+  p = fmaf(p, t, -1.13520398f);
+  p = fmaf(p, t, 0.27886807f);
+  p = fmaf(p, t, -0.18628806f);
+  p = fmaf(p, t, 0.09678418f);
+  p = fmaf(p, t, 0.37409196f);
+  p = fmaf(p, t, 1.00002368f);
+  p = fmaf(p, t, -1.26551223f);
+  const float half_erfc = 0.5f * t * __expf(fmaf(-z, z, p));
+  const float Phi = x >= 0.0f ? 1.0f - half_erfc : half_erfc;
+  const float dens = 0.39894228040143268f * __expf(-0.5f * x * x);
+  grad = fmaf(x, dens, Phi);
+  return x * Phi;
+}
+
+// act(v) and act'(v) for the backward's recomputation of the column layer.
+__device__ __forceinline__ float act_and_grad(float v, int act, float& grad) {
+  if (act == ACT_GELU) return gelu_and_grad(v, grad);
+  if (act == ACT_RELU) {
+    grad = v > 0.0f ? 1.0f : 0.0f;
+    return fmaxf(v, 0.0f);
+  }
+  grad = 1.0f;
+  return v;
 }
 
 // The element-wise nonlinearity of the column layer (ACT_NONE / ACT_GELU / ACT_RELU).

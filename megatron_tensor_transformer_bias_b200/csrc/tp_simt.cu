@@ -6,11 +6,18 @@
 //    on feature reductions: mean and variance need every feature), one CTA per
 //    row, row cached in shared memory, warp-shuffle reductions;
 //  * the exact-fp32 FFN (FFMA, no TF32) used for fp32 inputs;
+//  * column sums in a fixed order (the bias gradients of the backward pass);
 //  * the bounded-wait self-test kernel.
 #include "tp_internal.h"
 #include "tp_ptx.cuh"
 
 namespace tpb {
+
+#define TP_TRY_LAUNCH(expr)            \
+  do {                                 \
+    tp_status _s = (expr);             \
+    if (_s != TP_OK) return _s;        \
+  } while (0)
 
 namespace {
 
@@ -90,7 +97,8 @@ template <bool IN_F32, bool OUT_F16>
 __global__ void __launch_bounds__(LN_THREADS) layernorm_kernel(const void* __restrict__ x,
                                                                const uint16_t* __restrict__ g,
                                                                const uint16_t* __restrict__ b, int64_t h,
-                                                               float eps, uint16_t* __restrict__ y) {
+                                                               float eps, uint16_t* __restrict__ y,
+                                                               uint32_t* status) {
   extern __shared__ float row[];
   __shared__ float red[LN_THREADS / 32];
   const int64_t r = blockIdx.x;
@@ -137,6 +145,10 @@ __global__ void __launch_bounds__(LN_THREADS) layernorm_kernel(const void* __res
     }
     uint4 u;
     if (OUT_F16) {
+      float m = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(o[j]));
+      note_f16_range(status, m, DEV_RANGE_LAYERNORM);
       u.x = pack_f16x2(o[0], o[1]);
       u.y = pack_f16x2(o[2], o[3]);
       u.z = pack_f16x2(o[4], o[5]);
@@ -200,6 +212,56 @@ __global__ void __launch_bounds__(256) act_kernel(const float* __restrict__ x, f
     y[i] = act_apply(x[i], act);
 }
 
+// ---------------------------------------------------------------- column sums
+// out[c] = sum over rows of x[r, c] for a bf16 x [M, ld], in a fixed order: pass 1 gives
+// each 128-row chunk's sum per column (warp w of a CTA adds the chunk's rows w, w + 8, ...
+// in turn, then the 8 warps' sums are added in the order 0..7); pass 2 adds the chunks'
+// sums in the order 0, 1, ...  Each thread of pass 1 owns 8 adjacent columns (one
+// 16-byte load per row), so a warp reads 512 contiguous bytes of a row.
+constexpr int CS_ROWS = 128;
+constexpr int CS_COLS = 256;   // 32 lanes x 8 columns
+
+__global__ void __launch_bounds__(256) colsum_chunk_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t n,
+                                                           int64_t ld, float* __restrict__ part) {
+  __shared__ float red[8][CS_COLS];
+  const int w = threadIdx.x / 32, l = threadIdx.x % 32;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * CS_COLS + l * 8;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * CS_ROWS;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  pdl_wait();
+  if (c0 < n) {
+    for (int64_t r = r0 + w; r < r0 + CS_ROWS && r < M; r += 8) {
+      float f[8];
+      load_bf16x8(x + r * ld + c0, f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] += f[j];
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) red[w][l * 8 + j] = acc[j];
+  __syncthreads();
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * CS_COLS + threadIdx.x;
+  if (c < n) {
+    float v = red[0][threadIdx.x];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) v += red[i][threadIdx.x];
+    part[static_cast<int64_t>(blockIdx.y) * n + c] = v;
+  }
+  pdl_launch_dependents();
+}
+
+__global__ void __launch_bounds__(256) colsum_final_kernel(const float* __restrict__ part, int chunks, int64_t n,
+                                                           float* __restrict__ out) {
+  pdl_wait();
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (c < n) {
+    float v = part[c];
+    for (int i = 1; i < chunks; ++i) v += part[static_cast<int64_t>(i) * n + c];
+    out[c] = v;
+  }
+  pdl_launch_dependents();
+}
+
 // ---------------------------------------------------------------- self-test
 __global__ void selftest_wait_kernel(uint64_t limit_ns, uint32_t* status) {
   __shared__ uint64_t bar;
@@ -257,7 +319,8 @@ template <bool IN_F32, bool OUT_F16, int NCH>
 __global__ void __launch_bounds__(LN_THREADS) layernorm_reg_kernel(const void* __restrict__ x,
                                                                    const uint16_t* __restrict__ g,
                                                                    const uint16_t* __restrict__ b, int64_t h,
-                                                                   float eps, uint16_t* __restrict__ y) {
+                                                                   float eps, uint16_t* __restrict__ y,
+                                                                   uint32_t* status) {
   __shared__ float red[LN_THREADS / 32];
   const int64_t r = blockIdx.x;
   const int n8 = static_cast<int>(h / 8);
@@ -327,6 +390,10 @@ __global__ void __launch_bounds__(LN_THREADS) layernorm_reg_kernel(const void* _
     for (int j = 0; j < 8; ++j) o[j] = (f[k][j] - mean) * rstd * gg[j] + bb[j];
     uint4 u;
     if (OUT_F16) {
+      float m = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(o[j]));
+      note_f16_range(status, m, DEV_RANGE_LAYERNORM);
       u.x = pack_f16x2(o[0], o[1]); u.y = pack_f16x2(o[2], o[3]);
       u.z = pack_f16x2(o[4], o[5]); u.w = pack_f16x2(o[6], o[7]);
     } else {
@@ -342,7 +409,7 @@ template <int NCH>
 static tp_status launch_layernorm_reg(const void* x, int in_fp32, const void* g, const void* b, int64_t M, int64_t h,
                                       float eps, void* y, int out_f16, cudaStream_t stream) {
   const int key = (in_fp32 ? 1 : 0) | (out_f16 ? 2 : 0);
-  void (*kern)(const void*, const uint16_t*, const uint16_t*, int64_t, float, uint16_t*) =
+  void (*kern)(const void*, const uint16_t*, const uint16_t*, int64_t, float, uint16_t*, uint32_t*) =
       key == 0   ? layernorm_reg_kernel<false, false, NCH>
       : key == 1 ? layernorm_reg_kernel<true, false, NCH>
       : key == 2 ? layernorm_reg_kernel<false, true, NCH>
@@ -350,7 +417,7 @@ static tp_status launch_layernorm_reg(const void* x, int in_fp32, const void* g,
   trace_before(stream);
   const tp_status st = launch_ex(kern, dim3(static_cast<unsigned>(M)), dim3(LN_THREADS), 0, stream, 1, x,
                                  static_cast<const uint16_t*>(g), static_cast<const uint16_t*>(b), h, eps,
-                                 static_cast<uint16_t*>(y));
+                                 static_cast<uint16_t*>(y), device_status_ptr());
   if (st != TP_OK) return st;
   trace_after(stream, "layernorm");
   return TP_OK;
@@ -366,7 +433,7 @@ tp_status launch_layernorm(const void* x, int in_fp32, const void* g, const void
   if (M == 0) return TP_OK;
   const size_t smem = static_cast<size_t>(h) * sizeof(float);
   const int key = (in_fp32 ? 1 : 0) | (out_f16 ? 2 : 0);
-  void (*kern)(const void*, const uint16_t*, const uint16_t*, int64_t, float, uint16_t*) =
+  void (*kern)(const void*, const uint16_t*, const uint16_t*, int64_t, float, uint16_t*, uint32_t*) =
       key == 0 ? layernorm_kernel<false, false>
                : key == 1 ? layernorm_kernel<true, false> : key == 2 ? layernorm_kernel<false, true>
                                                                      : layernorm_kernel<true, true>;
@@ -381,7 +448,7 @@ tp_status launch_layernorm(const void* x, int in_fp32, const void* g, const void
   trace_before(stream);
   const tp_status st = launch_ex(kern, dim3(static_cast<unsigned>(M)), dim3(LN_THREADS), smem, stream, 1, x,
                                  static_cast<const uint16_t*>(g), static_cast<const uint16_t*>(b), h, eps,
-                                 static_cast<uint16_t*>(y));
+                                 static_cast<uint16_t*>(y), device_status_ptr());
   if (st != TP_OK) return st;
   trace_after(stream, "layernorm");
   return TP_OK;
@@ -428,6 +495,29 @@ tp_status launch_act(const float* x, float* y, int64_t n, int act, cudaStream_t 
   act_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(x, y, n, act);
   if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
   trace_after(stream, "activation");
+  return TP_OK;
+}
+
+size_t colsum_workspace_bytes(int64_t M, int64_t n) {
+  return static_cast<size_t>((M + CS_ROWS - 1) / CS_ROWS) * static_cast<size_t>(n) * sizeof(float);
+}
+
+tp_status launch_colsum(const void* x, int64_t M, int64_t n, int64_t ld, float* part, float* out,
+                        cudaStream_t stream) {
+  if (n == 0) return TP_OK;
+  const int chunks = static_cast<int>((M + CS_ROWS - 1) / CS_ROWS);
+  if (chunks == 0) {
+    const cudaError_t e = cudaMemsetAsync(out, 0, static_cast<size_t>(n) * sizeof(float), stream);
+    return e == cudaSuccess ? TP_OK : set_error(TP_ERR_CUDA, cudaGetErrorString(e));
+  }
+  trace_before(stream);
+  TP_TRY_LAUNCH(launch_ex(colsum_chunk_kernel, dim3(static_cast<unsigned>((n + CS_COLS - 1) / CS_COLS), chunks),
+                          dim3(256), 0, stream, 1, static_cast<const uint16_t*>(x), M, n, ld, part));
+  trace_after(stream, "colsum");
+  trace_before(stream);
+  TP_TRY_LAUNCH(launch_ex(colsum_final_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, stream, 1,
+                          static_cast<const float*>(part), chunks, n, out));
+  trace_after(stream, "colsum");
   return TP_OK;
 }
 

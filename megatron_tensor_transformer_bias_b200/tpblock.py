@@ -16,7 +16,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libtpblock.so")
 
-TP_OK, TP_ERR_INVALID_ARG, TP_ERR_UNSUPPORTED, TP_ERR_WORKSPACE, TP_ERR_CUDA, TP_ERR_TIMEOUT = range(6)
+TP_OK, TP_ERR_INVALID_ARG, TP_ERR_UNSUPPORTED, TP_ERR_WORKSPACE, TP_ERR_CUDA, TP_ERR_TIMEOUT, TP_ERR_RANGE = range(7)
 TP_BF16, TP_FP32, TP_FP16 = 0, 1, 2
 TP_REDUCE_FUSED, TP_REDUCE_PARTIALS = 0, 1
 TP_ACT_GELU, TP_ACT_RELU = 0, 1
@@ -49,6 +49,9 @@ _SIGS = {
     "tp_ffn_forward_act": (_i32, [_vp, _i64, _i64, _i64, _i32, _SP, _VPP, _SP, _vp, _vp, _vp, _i32, _i32, _i32, _vp,
                                   _sz, _vp]),
     "tp_ffn_forward_noalloc": (_i32, [_vp, _i64, _i64, _i64, _i32, _SP, _VPP, _SP, _vp, _vp, _vp, _vp]),
+    "tp_ffn_backward_workspace_bytes": (_sz, [_i64, _i64, _i64, _i32]),
+    "tp_ffn_backward": (_i32, [_vp, _i64, _i64, _i64, _i32, _SP, _VPP, _SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
+                               _vp, _sz, _vp]),
     "tp_column_linear_forward": (_i32, [_vp, _i64, _i64, _i64, _i32, _SP, _VPP, _i32, _vp, _vp]),
     "tp_row_linear_workspace_bytes": (_sz, [_i64, _i64, _i32, _i32]),
     "tp_row_linear_forward": (_i32, [_vp, _i64, _i64, _i64, _i32, _SP, _vp, _vp, _vp, _i32, _vp, _sz, _vp]),
@@ -209,6 +212,29 @@ def tp_ffn_forward_noalloc(X, W1, b1, W2, b2, residual, out, stream=None):
     _check(lib().tp_ffn_forward_noalloc(_ptr(X), M, h, f, t, _shards(W1), _ptr_array(b1), _shards(W2), _ptr(b2),
                                         _ptr(residual), _ptr(out), _stream(stream)))
     return out
+
+
+def tp_ffn_backward_workspace_bytes(M, h, f, t) -> int:
+    return lib().tp_ffn_backward_workspace_bytes(M, h, f, t)
+
+
+def tp_ffn_backward(X, W1, b1, W2, dY, dX, dW1, dW2, db1=None, db2=None, dX_add=None, act="gelu", ws=None,
+                    stream=None):
+    """Gradients of the FFN block (bf16): dX [M,h] bf16, dW1 [h,f] fp32, dW2 [f,h] fp32,
+    db1 [f] and db2 [h] fp32 (optional), for the upstream gradient dY [M,h] bf16."""
+    for t_ in (X, dY, dX, dW1, dW2):
+        _dev(t_)
+    M, h = X.shape
+    t = len(W1)
+    f = sum(w.shape[1] for w in W1)
+    if dW1.dtype != torch.float32 or dW2.dtype != torch.float32:
+        raise ValueError("weight gradients are fp32")
+    if ws is None:
+        ws = workspace(tp_ffn_backward_workspace_bytes(M, h, f, t), X.device)
+    _check(lib().tp_ffn_backward(_ptr(X), M, h, f, t, _shards(W1), _ptr_array(b1), _shards(W2), _ptr(dY),
+                                 _ptr(dX_add), _ptr(dX), _ptr(dW1), _ptr(db1), _ptr(dW2), _ptr(db2), ACTS[act],
+                                 _ptr(ws), ws.numel(), _stream(stream)))
+    return dX, dW1, dW2, db1, db2
 
 
 def tp_column_linear_forward(X, W, b, out, act=None, stream=None):

@@ -46,11 +46,15 @@ def test_workspace_sizes(L):
     M, h, f, t = 2048, 4096, 16384, 4
     z = M * f * 2
     assert tb.tp_ffn_workspace_bytes(M, h, f, t, tb.TP_BF16, tb.TP_REDUCE_FUSED) == z
-    assert tb.tp_ffn_workspace_bytes(M, h, f, t, tb.TP_BF16, tb.TP_REDUCE_PARTIALS) == z + t * M * h * 4
+    ctr = ((M + 31) // 32) * ((h + 127) // 128) * 4          # arrival counters of the in-epilogue reduction
+    assert tb.tp_ffn_workspace_bytes(M, h, f, t, tb.TP_BF16, tb.TP_REDUCE_PARTIALS) == z + t * M * h * 4 + ctr
     assert tb.tp_ffn_workspace_bytes(8, 64, 256, 2, tb.TP_FP32, tb.TP_REDUCE_FUSED) == 8 * 256 * 4 + 2 * 8 * 64 * 4
     assert tb.tp_ffn_workspace_bytes(0, h, f, t) == 0
     assert L.tp_row_linear_workspace_bytes(M, h, t, tb.TP_REDUCE_FUSED) == 0
-    assert L.tp_row_linear_workspace_bytes(M, h, t, tb.TP_REDUCE_PARTIALS) == t * M * h * 4
+    assert L.tp_row_linear_workspace_bytes(M, h, t, tb.TP_REDUCE_PARTIALS) == t * M * h * 4 + ctr
+    mf = M * f * 2
+    assert tb.tp_ffn_backward_workspace_bytes(M, h, f, t) == 3 * mf + (M + 127) // 128 * f * 4
+    assert tb.tp_ffn_backward_workspace_bytes(0, h, f, t) == 0
     B, S, H, d = 2, 2048, 32, 128
     q = B * S * H * d * 2
     assert tb.tp_attn_workspace_bytes(B, S, 4096, H, d, 4, tb.TP_REDUCE_FUSED) == 4 * q
@@ -169,3 +173,22 @@ def test_binding_requires_library(monkeypatch):
     monkeypatch.setattr(tb, "LIB_PATH", "/nonexistent/libtpblock.so")
     with pytest.raises(RuntimeError, match="not built"):
         tb.lib()
+
+
+def test_backward_validation(L):
+    M, h, f, t = 256, 256, 1024, 2
+
+    def call(**k):
+        return L.tp_ffn_backward(k.get("X", FAKE), k.get("M", M), h, k.get("f", f), t, k.get("W1", _sh(t, f)), None,
+                                 k.get("W2", _sh(t, h)), k.get("dY", FAKE + 8192), None, k.get("dX", FAKE + 4096),
+                                 k.get("dW1", FAKE + 16384), None, k.get("dW2", FAKE + 32768), None,
+                                 k.get("act", tb.TP_ACT_GELU), k.get("ws", FAKE), 0, None)
+    assert call(dY=None) == tb.TP_ERR_INVALID_ARG and "dY is NULL" in tb.last_error()
+    assert call(dW1=None) == tb.TP_ERR_INVALID_ARG and "dW1 is NULL" in tb.last_error()
+    assert call(dX=FAKE) == tb.TP_ERR_INVALID_ARG and "alias" in tb.last_error()
+    assert call(act=5) == tb.TP_ERR_INVALID_ARG and "activation" in tb.last_error()
+    assert call(f=1001) == tb.TP_ERR_INVALID_ARG and "divisible" in tb.last_error()
+    w2 = _sh(t, h)
+    w2[0].dtype = w2[1].dtype = tb.TP_FP16
+    assert call(W2=w2) == tb.TP_ERR_UNSUPPORTED and "bf16" in tb.last_error()
+    assert call() == tb.TP_ERR_WORKSPACE and "workspace" in tb.last_error()

@@ -53,11 +53,34 @@ def test_reference_arm_runs_on_cpu(capsys, monkeypatch):
     import json
     import sys
     import bench
-    monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--steps", "2", "--warmup", "3"])
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--workload", "ffn", "--steps", "2",
+                                      "--warmup", "3"])
     bench.main()
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["cpu_baseline"]["host_cpus"] == os.cpu_count() and "cores" in line["cpu_baseline"]
+
+
+def test_reference_arm_tiny_fp32_and_workload_order(capsys, monkeypatch):
+    """The default workload list ends with the headline FFN block; the tiny fp32 block's
+    reference line runs the oracle on all 8 rows per step."""
+    import json
+    import sys
+    import bench
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--workload", "fp32", "--steps", "2",
+                                      "--warmup", "3"])
+    bench.main()
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["config"]["workload"] == "ffn_fp32_M8_h64_f256_t2" and line["value"] > 0
+
+    class A:
+        workload, impl, mode, t, h = "all", "ours", "fused", 4, "22528"
+    names = [w.name for w in bench.make_workloads(A)]
+    assert names[-1] == "ffn_bf16_M2048_h4096_f16384_t4" and len(names) == len(set(names)) == 8
+    assert "ffn_bwd_bf16_M2048_h4096_f16384_t4" in names
+    A.impl = "reference"
+    assert bench.make_workloads(A)[-1].headline
 
 
 def test_kernel_source_hash_ignores_comments_only():

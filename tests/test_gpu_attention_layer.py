@@ -133,3 +133,25 @@ def test_layer_S2048_h8192_sampled():
     assert torch.isfinite(out.float()).all()
     del p
     torch.cuda.empty_cache()
+
+
+def test_layer_S2048_h8192_bf16_weights_error_recorded():
+    """The full layer with the bf16 weights as given (LN1/LN2 outputs, O and act(Z)
+    in bf16; Q, K, V, P stay fp16).  Records the measured error against the oracle
+    (prefix RECORD) next to the fp16-weight run; asserts only finiteness, since
+    the relative Frobenius bound is what bf16 intermediates break here."""
+    from tests.parity import errors
+    w = configs.LAYER_S2048_H8192
+    p = inputs.layer_inputs(w.B, w.S, w.h, w.H, w.d, w.f, seed=0, device=DEV)
+    rows = inputs.sample_rows(w.M, configs.SAMPLED_ROWS, seq=w.S)
+    ref = _layer_ref(p, w.B, w.S, w.H, w.d, True, rows=rows)
+    out = _layer_gpu(p, w.B, w.S, w.H, w.d, w.t, fp16=False)
+    rel_fro, excess, maxabs = errors(out[rows], ref)
+    out16 = _layer_gpu(p, w.B, w.S, w.H, w.d, w.t, fp16=True)
+    rel16, excess16, maxabs16 = errors(out16[rows], ref)
+    print(f"RECORD layer h=8192: bf16 weights rel_fro={rel_fro:.3e} max|err|={maxabs:.3e} "
+          f"element_excess={excess:.3e}; fp16 weights rel_fro={rel16:.3e} max|err|={maxabs16:.3e} "
+          f"element_excess={excess16:.3e}")
+    assert torch.isfinite(out.float()).all()
+    del p
+    torch.cuda.empty_cache()

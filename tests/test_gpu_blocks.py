@@ -81,7 +81,8 @@ def test_launch_trace_names_kernels():
     finally:
         tb.tp_trace_disable()
     names = [n for n, _ in recs]
-    assert names == ["gemm_column_act", "gemm_row_partials", "reduce_partials"]
+    # partials mode: the last shard's tiles sum the partials inside the row GEMM
+    assert names == ["gemm_column_act", "gemm_row_partials"]
     assert all(ms > 0 for _, ms in recs)
 
 

@@ -2,6 +2,8 @@
 
 Small cases compare every element; full-size workloads compare a seeded sample
 of 64 token rows.  All calls go through the C-ABI (ctypes binding)."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -13,6 +15,7 @@ from tests.parity import assert_bf16_close, assert_fp32_close, ffn_oracle_rows, 
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _run_ffn(inp, t, mode="fused", act="gelu", with_b1=True, with_b2=True, with_res=True, w2_fp16=False):
@@ -139,6 +142,55 @@ def test_row_linear(mode):
     assert_bf16_close(out, ref, f"row linear {mode}")
 
 
+ROW_PARTIAL_CASES = [(300, 384, 4), (1, 320, 2), (129, 256, 1), (513, 1024, 8), (2048, 4096, 4)]
+
+
+def _row_partials_case(M, n, t):
+    k = 256 * t
+    g = torch.Generator(device=DEV).manual_seed(M + n + t)
+    A = torch.randn(M, k, generator=g, device=DEV).to(torch.bfloat16)
+    W = (torch.randn(k, n, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    bias = (torch.randn(n, generator=g, device=DEV) * 0.01).to(torch.bfloat16)
+    R = torch.randn(M, n, generator=g, device=DEV).to(torch.bfloat16)
+    ws = tb.workspace(tb.lib().tp_row_linear_workspace_bytes(M, n, t, tb.TP_REDUCE_PARTIALS), DEV)
+    out = torch.empty(M, n, dtype=torch.bfloat16, device=DEV)
+    runs = []
+    for _ in range(2):
+        out.fill_(float("nan"))
+        tb.tp_row_linear_forward(A, tb.shard_rows(W, t), bias, R, out, mode="partials", ws=ws)
+        assert tb.tp_get_device_status() == tb.TP_OK
+        runs.append(out.clone())
+    P = ws[: t * M * n * 4].view(torch.float32).view(t, M, n)[: t - 1].clone()
+    return runs, P
+
+
+def test_row_partials_reduce_matches_separate_pass(tmp_path):
+    """Partials mode sums each region's t partials inside the row GEMM (the last shard's
+    tiles add the stored partials 0..t-2 and their own, in order 0..t-1).  The output must
+    be the same bits as summing the stored partials in a separate pass afterwards, which a
+    child process runs with TPB_SEPARATE_REDUCE=1 on the same inputs; the partials 0..t-2
+    left in the workspace must match too, and two calls in a row must agree (the arrival
+    counters start from zero every call)."""
+    import subprocess
+    import sys
+    here = {}
+    for case in ROW_PARTIAL_CASES:
+        runs, P = _row_partials_case(*case)
+        assert torch.equal(runs[0], runs[1]), case
+        here[case] = (runs[0].cpu(), P.cpu())
+    dump = tmp_path / "separate.pt"
+    code = ("import sys, torch; sys.path.insert(0, %r); from tests import test_gpu_ffn as T; "
+            "torch.save({c: tuple(x.cpu() for x in (T._row_partials_case(*c)[0][0], T._row_partials_case(*c)[1])) "
+            "for c in T.ROW_PARTIAL_CASES}, %r)" % (ROOT, str(dump)))
+    r = subprocess.run([sys.executable, "-c", code], env=dict(os.environ, TPB_SEPARATE_REDUCE="1"),
+                       capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-3000:]
+    there = torch.load(dump)
+    for case in ROW_PARTIAL_CASES:
+        assert torch.equal(here[case][0], there[case][0]), f"output {case}"
+        assert torch.equal(here[case][1], there[case][1]), f"partials {case}"
+
+
 # ---------------------------------------------------------------- full-size workloads (sampled rows)
 @pytest.fixture(scope="module")
 def ffn_2048():
@@ -182,6 +234,31 @@ def test_ffn_hidden_sweep_sampled(h):
         out = _run_ffn(inp, t, w2_fp16=True)
         assert_bf16_close(out[rows], ref, f"M4096 h{h} t{t}")
     del inp, out
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("h", [8192, 22528])
+def test_ffn_hidden_sweep_bf16_w2_error_recorded(h):
+    """The same sweep points with bf16 W2 (act(Z) stored in bf16), the deviation the
+    fp16 copy avoids.  Records the measured error against the oracle (printed with
+    the prefix RECORD); asserts only the relative Frobenius bound, which holds, while
+    the per-element bound 3e-2 + 2e-2|ref| is what bf16 act(Z) breaks at these sizes."""
+    from tests.parity import errors
+    M = 4096
+    inp = inputs.ffn_inputs(M, h, 4 * h, "bf16", seed=0, device=DEV)
+    rows = inputs.sample_rows(M, configs.SAMPLED_ROWS)
+    ref = ffn_oracle_rows(inp, rows, chunks=16)
+    for t in configs.SWEEP_SHARDS:
+        out = _run_ffn(inp, t, w2_fp16=False)
+        rel_fro, excess, maxabs = errors(out[rows], ref)
+        out16 = _run_ffn(inp, t, w2_fp16=True)
+        rel16, excess16, maxabs16 = errors(out16[rows], ref)
+        print(f"RECORD sweep h={h} t={t}: bf16 act(Z) rel_fro={rel_fro:.3e} max|err|={maxabs:.3e} "
+              f"element_excess={excess:.3e}; fp16 act(Z) rel_fro={rel16:.3e} max|err|={maxabs16:.3e} "
+              f"element_excess={excess16:.3e}")
+        assert rel_fro <= 5e-3
+        assert excess16 <= 0
+    del inp, out, out16
     torch.cuda.empty_cache()
 
 
