@@ -43,6 +43,10 @@ constexpr int THREADS = 64 + 32 * EPI_WARPS;        // warp 0 TMA, warp 1 MMA, w
 constexpr int STAGING_BYTES = EPI_WARPS * 2 * 2048;   // two 32x32 16-bit buffers per epilogue warp
 constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + 256;
 
+// Operand layouts a kernel instantiation is compiled for (template parameter OPL).
+constexpr int OPL_A_MN = 1;      // A M-major (the backward's weight gradients)
+constexpr int OPL_B_KMAJOR = 2;  // B K-major (the backward's input gradients)
+
 struct TileCoord {
   int g, m_blk, n_blk;
 };
@@ -125,15 +129,16 @@ __device__ __forceinline__ void store_x32(void* base, int64_t idx, int out_type,
 // Bias / nonlinearity / residual of one 32-column chunk for the epilogues whose
 // 16-bit output leaves through a TMA store (EPI_ACT, EPI_BIAS_RESID).  Rows at or
 // beyond M still run (their values are clipped by the store) but read no residual.
+template <int EPI>
 __device__ __forceinline__ void epilogue_math(const GemmArgs& a, const TileCoord& tc, int row, int n, float (&v)[32]) {
-  const void* bias = a.epi == EPI_ACT ? a.bias_g[tc.g] : a.bias;
+  const void* bias = EPI == EPI_ACT ? a.bias_g[tc.g] : a.bias;
   if (bias) {
     float b[32];
     load_bf16x32(static_cast<const uint16_t*>(bias) + n, b);
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] += b[j];
   }
-  if (a.epi == EPI_ACT) {
+  if (EPI == EPI_ACT) {
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = act_apply(v[j], a.act);
   } else if (a.resid && row < a.M) {
@@ -200,10 +205,11 @@ __device__ __forceinline__ void load_f16x32(const void* p, float (&v)[32]) {
 
 // One 32-column chunk of an epilogue whose 16-bit output leaves through TMA stores.
 // `x` is the chunk's first output column, `y0` the first row of the warp's 32 rows.
+template <int EPI>
 __device__ __forceinline__ void epilogue_tma_chunk(const GemmArgs& a, const TileCoord& tc, int row, int n,
                                                    float (&v)[32], uint8_t* warp_staging, int& count, int lane,
                                                    int x, int y0) {
-  if (a.epi == EPI_ACT_GRAD) {
+  if (EPI == EPI_ACT_GRAD) {
     // the backward's recomputation of the column layer: act(z) and act'(z), z = acc + b
     if (a.bias_g[tc.g]) {
       float b[32];
@@ -218,7 +224,7 @@ __device__ __forceinline__ void epilogue_tma_chunk(const GemmArgs& a, const Tile
     stage_and_store(a, &a.tmOut2, OUT_F16, warp_staging, count, lane, gr, x, y0);
     return;
   }
-  if (a.epi == EPI_MUL_GRAD) {
+  if (EPI == EPI_MUL_GRAD) {
     // dZ = dA * act'(Z): the factor sits at the output's own position
     if (row < a.M) {
       float gm[32];
@@ -229,7 +235,7 @@ __device__ __forceinline__ void epilogue_tma_chunk(const GemmArgs& a, const Tile
     stage_and_store(a, &a.tmOut, a.out_type, warp_staging, count, lane, v, x, y0);
     return;
   }
-  epilogue_math(a, tc, row, n, v);
+  epilogue_math<EPI>(a, tc, row, n, v);
   stage_and_store(a, &a.tmOut, a.out_type, warp_staging, count, lane, v, x, y0);
 }
 
@@ -350,9 +356,10 @@ __device__ __forceinline__ void reduce_chunk(const GemmArgs& a, int row, int n, 
 }
 
 // One 32-column chunk of one accumulator row: apply the epilogue and store.
+template <int EPI>
 __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, const TileCoord& tc, int row, int n,
                                                float (&v)[32]) {
-  switch (a.epi) {
+  switch (EPI) {
     case EPI_ACT: {
       if (a.bias_g[tc.g]) {
         float b[32];
@@ -418,7 +425,10 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& a, const TileCoor
   }
 }
 
+template <int EPI, int OPL>
 __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_constant__ GemmArgs a) {
+  constexpr bool A_MN = (OPL & OPL_A_MN) != 0;
+  constexpr bool B_KM = (OPL & OPL_B_KMAJOR) != 0;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte-swizzled tiles.
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -495,13 +505,13 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
           mbar_arrive_expect_tx(&full_bar[stage], STAGE_BYTES);
           uint8_t* a_dst = sA + stage * A_STAGE_BYTES;
           const int ka = g * a.a_k_per_group + kb * BK;
-          if (!a.a_mn) {
+          if (!A_MN) {
             tma_load_2d_hint(a_dst, &a.tmA, &full_bar[stage], ka, m0, pol_a);
           } else {  // two 64-wide M blocks of 64 K rows
             tma_load_3d_hint(a_dst, &a.tmA, &full_bar[stage], 0, ka, (g * a.a_m_per_group + m0) / 64, pol_a);
           }
           uint8_t* b_dst = sB + stage * B_STAGE_BYTES;
-          if (!a.b_kmajor) {  // four 64-wide N blocks of 64 K rows, two per load
+          if (!B_KM) {  // four 64-wide N blocks of 64 K rows, two per load
             tma_load_3d_hint(b_dst, &a.tmB[g], &full_bar[stage], 0, kb * BK, n0 / 64, pol_b);
             tma_load_3d_hint(b_dst + 2 * B_BLOCK_BYTES, &a.tmB[g], &full_bar[stage], 0, kb * BK, n0 / 64 + 2, pol_b);
           } else {  // two 128-row N blocks of 64 K each
@@ -529,8 +539,8 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      const uint32_t idesc = a.ab_f16 ? idesc_f16_f32(BM, BN, a.a_mn, !a.b_kmajor)
-                                      : idesc_bf16_f32(BM, BN, a.a_mn, !a.b_kmajor);
+      const uint32_t idesc = a.ab_f16 ? idesc_f16_f32(BM, BN, A_MN, !B_KM)
+                                      : idesc_bf16_f32(BM, BN, A_MN, !B_KM);
       const uint32_t sA_addr = smem_u32(sA);
       const uint32_t sB_addr = smem_u32(sB);
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
@@ -551,9 +561,9 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
           for (int k = 0; k < BK / 16; ++k) {
             // K-major operand: advance 16 elements (32 bytes) inside the swizzle atom;
             // MN-major operand: advance 16 K-rows (2048 bytes), 64-wide MN blocks 8 KB apart.
-            const uint64_t adesc = a.a_mn ? smem_desc_sw128(a_base + k * 16 * 128, B_BLOCK_BYTES, 1024)
+            const uint64_t adesc = A_MN ? smem_desc_sw128(a_base + k * 16 * 128, B_BLOCK_BYTES, 1024)
                                           : smem_desc_sw128(a_base + k * 32, 16, 1024);
-            const uint64_t bdesc = a.b_kmajor ? smem_desc_sw128(b_base + k * 32, 16, 1024)
+            const uint64_t bdesc = B_KM ? smem_desc_sw128(b_base + k * 32, 16, 1024)
                                               : smem_desc_sw128(b_base + k * 16 * 128, B_BLOCK_BYTES, 1024);
             mma_bf16_ss(d_tmem, adesc, bdesc, idesc, (it > 0 || k > 0) ? 1u : 0u);
           }
@@ -575,8 +585,8 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
     const int col_half = (warp - 2) / 4;    // columns [col_half*BN/2, +BN/2) of each tile
     int acc = 0;
     uint32_t acc_phase = 0;
-    const bool tma_out = a.tma_store && (a.epi == EPI_ACT || a.epi == EPI_BIAS_RESID || a.epi == EPI_ACT_GRAD ||
-                                         a.epi == EPI_MUL_GRAD);
+    const bool tma_out = a.tma_store && (EPI == EPI_ACT || EPI == EPI_BIAS_RESID || EPI == EPI_ACT_GRAD ||
+                                         EPI == EPI_MUL_GRAD);
     uint8_t* warp_staging = staging + (warp - 2) * 4096;
     int store_count = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -601,9 +611,9 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
       if (n0 + c_end * 32 > a.N) c_end = (a.N - n0) / 32;
       // partials mode with the reduction here: this warp's region and its role in it
       const int row0 = tc.m_blk * BM + sub * 32;
-      const bool in_region = a.red_out && row0 < a.M && c_begin < c_end;
+      const bool in_region = EPI == EPI_PARTIAL_F32 && a.red_out && row0 < a.M && c_begin < c_end;
       const int ctr = in_region ? region_counter(a, row0, n0 / 128 + col_half) : 0;
-      const bool red_tile = a.red_out && tc.g == a.G - 1;
+      const bool red_tile = EPI == EPI_PARTIAL_F32 && a.red_out && tc.g == a.G - 1;
       bool red_ok = true;
       if (red_tile && in_region) {
         red_ok = partial_wait(a, ctr, lane);
@@ -624,10 +634,10 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
           if (red_tile) {
             reduce_chunk(a, row, n0 + c * 32, v, red_ok, warp_staging, store_count, lane);
           } else if (tma_out) {
-            const int x = (a.epi == EPI_BIAS_RESID ? 0 : tc.g * static_cast<int>(a.out_col_per_group)) + n0 + c * 32;
-            epilogue_tma_chunk(a, tc, row, n0 + c * 32, v, warp_staging, store_count, lane, x, row - lane);
+            const int x = (EPI == EPI_BIAS_RESID ? 0 : tc.g * static_cast<int>(a.out_col_per_group)) + n0 + c * 32;
+            epilogue_tma_chunk<EPI>(a, tc, row, n0 + c * 32, v, warp_staging, store_count, lane, x, row - lane);
           } else if (row < a.M) {
-            epilogue_chunk(a, tc, row, n0 + c * 32, v);
+            epilogue_chunk<EPI>(a, tc, row, n0 + c * 32, v);
           }
         }
         tmem_ld_wait();
@@ -667,7 +677,10 @@ constexpr int P_B_BYTES = (BN / 2) * BK * 2;        // 16 KB per CTA
 constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
 constexpr int P_SMEM_BYTES = 1024 + P_STAGES * P_STAGE_BYTES + STAGING_BYTES + 256;
 
+template <int EPI, int OPL>
 __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_constant__ GemmArgs a) {
+  constexpr bool A_MN = (OPL & OPL_A_MN) != 0;
+  constexpr bool B_KM = (OPL & OPL_B_KMAJOR) != 0;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -754,13 +767,13 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
           if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * P_STAGE_BYTES);
           uint8_t* a_dst = sA + stage * P_A_BYTES;
           const int ka = g * a.a_k_per_group + kb * BK;
-          if (!a.a_mn) {
+          if (!A_MN) {
             tma_load_2d_pair(a_dst, &a.tmA, fb, ka, m0, pol_a);
           } else {  // two 64-wide M blocks of 64 K rows, one load
             tma_load_3d_pair(a_dst, &a.tmA, fb, 0, ka, (g * a.a_m_per_group + m0) / 64, pol_a);
           }
           uint8_t* b_dst = sB + stage * P_B_BYTES;
-          if (!a.b_kmajor) {  // this CTA's two 64-wide N blocks of 64 K rows, one load
+          if (!B_KM) {  // this CTA's two 64-wide N blocks of 64 K rows, one load
             tma_load_3d_pair(b_dst, &a.tmB[g], fb, 0, kb * BK, n0 / 64, pol_b);
           } else {  // this CTA's 128 N rows, 64 K each
             tma_load_2d_pair(b_dst, &a.tmB[g], fb, kb * BK, n0, pol_b);
@@ -782,8 +795,8 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader only)
     if (lane == 0 && leader) {
-      const uint32_t idesc = a.ab_f16 ? idesc_f16_f32(P_ROWS, BN, a.a_mn, !a.b_kmajor)
-                                      : idesc_bf16_f32(P_ROWS, BN, a.a_mn, !a.b_kmajor);
+      const uint32_t idesc = a.ab_f16 ? idesc_f16_f32(P_ROWS, BN, A_MN, !B_KM)
+                                      : idesc_bf16_f32(P_ROWS, BN, A_MN, !B_KM);
       const uint32_t sA_addr = smem_u32(sA);
       const uint32_t sB_addr = smem_u32(sB);
       int stage = 0;
@@ -807,9 +820,9 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
           const uint32_t b_base = sB_addr + stage * P_B_BYTES;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
-            const uint64_t adesc = a.a_mn ? smem_desc_sw128(a_base + k * 16 * 128, B_BLOCK_BYTES, 1024)
+            const uint64_t adesc = A_MN ? smem_desc_sw128(a_base + k * 16 * 128, B_BLOCK_BYTES, 1024)
                                           : smem_desc_sw128(a_base + k * 32, 16, 1024);
-            const uint64_t bdesc = a.b_kmajor ? smem_desc_sw128(b_base + k * 32, 16, 1024)
+            const uint64_t bdesc = B_KM ? smem_desc_sw128(b_base + k * 32, 16, 1024)
                                               : smem_desc_sw128(b_base + k * 16 * 128, B_BLOCK_BYTES, 1024);
             mma_pair_ss(d_tmem, adesc, bdesc, idesc, (it > 0 || k > 0) ? 1u : 0u);
           }
@@ -831,8 +844,8 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
     const uint32_t acc_empty0_leader = mapa_shared(smem_u32(&acc_empty[0]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
-    const bool tma_out = a.tma_store && (a.epi == EPI_ACT || a.epi == EPI_BIAS_RESID || a.epi == EPI_ACT_GRAD ||
-                                         a.epi == EPI_MUL_GRAD);
+    const bool tma_out = a.tma_store && (EPI == EPI_ACT || EPI == EPI_BIAS_RESID || EPI == EPI_ACT_GRAD ||
+                                         EPI == EPI_MUL_GRAD);
     uint8_t* warp_staging = staging + (warp - 2) * 4096;
     int store_count = 0;
     for (int tile = cid; tile < num_tiles; tile += nclusters) {
@@ -856,9 +869,9 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
       if (n0 + c_end * 32 > a.N) c_end = (a.N - n0) / 32;
       // partials mode with the reduction here: this warp's region and its role in it
       const int row0 = tc.m_blk * P_ROWS + static_cast<int>(rank) * BM + sub * 32;
-      const bool in_region = a.red_out && row0 < a.M && c_begin < c_end;
+      const bool in_region = EPI == EPI_PARTIAL_F32 && a.red_out && row0 < a.M && c_begin < c_end;
       const int ctr = in_region ? region_counter(a, row0, n0 / 128 + col_half) : 0;
-      const bool red_tile = a.red_out && tc.g == a.G - 1;
+      const bool red_tile = EPI == EPI_PARTIAL_F32 && a.red_out && tc.g == a.G - 1;
       bool red_ok = true;
       if (red_tile && in_region) {
         red_ok = partial_wait(a, ctr, lane);
@@ -879,10 +892,10 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
           if (red_tile) {
             reduce_chunk(a, row, n0 + c * 32, v, red_ok, warp_staging, store_count, lane);
           } else if (tma_out) {
-            const int x = (a.epi == EPI_BIAS_RESID ? 0 : tc.g * static_cast<int>(a.out_col_per_group)) + n0 + c * 32;
-            epilogue_tma_chunk(a, tc, row, n0 + c * 32, v, warp_staging, store_count, lane, x, row - lane);
+            const int x = (EPI == EPI_BIAS_RESID ? 0 : tc.g * static_cast<int>(a.out_col_per_group)) + n0 + c * 32;
+            epilogue_tma_chunk<EPI>(a, tc, row, n0 + c * 32, v, warp_staging, store_count, lane, x, row - lane);
           } else if (row < a.M) {
-            epilogue_chunk(a, tc, row, n0 + c * 32, v);
+            epilogue_chunk<EPI>(a, tc, row, n0 + c * 32, v);
           }
         }
         tmem_ld_wait();
@@ -919,15 +932,54 @@ static bool gemm_use_pairs() {
   return v == 1;
 }
 
-static int g_pair_clusters[64] = {0};
+typedef void (*GemmKernel)(GemmArgs);
 
-// Largest number of co-resident CTA pairs for the pair kernel on this device.
+// The kernel instantiation for an epilogue kind and operand layout: each instantiation holds
+// only its own epilogue and operand addressing, so neither the register budget nor the
+// single MMA-issuing thread pays for the paths it does not take.  The combinations the
+// library launches: forward layers (K-major A, N-major B) with every forward epilogue; the
+// backward's dZ (K-major B, fp16 factor), weight gradients (M-major A, fp32 out) and dX
+// (K-major B, sum over shards).
+static GemmKernel gemm_kernel_for(int epi, int opl, bool pair) {
+#define TP_GEMM_PICK(E, O) \
+  if (epi == E && opl == O) return pair ? tp_gemm_pair_kernel<E, O> : tp_gemm_kernel<E, O>;
+  TP_GEMM_PICK(EPI_ACT, 0)
+  TP_GEMM_PICK(EPI_PARTIAL_F32, 0)
+  TP_GEMM_PICK(EPI_BIAS_RESID, 0)
+  TP_GEMM_PICK(EPI_QKV, 0)
+  TP_GEMM_PICK(EPI_ACT_GRAD, 0)
+  TP_GEMM_PICK(EPI_MUL_GRAD, OPL_B_KMAJOR)
+  TP_GEMM_PICK(EPI_PARTIAL_F32, OPL_A_MN)
+  TP_GEMM_PICK(EPI_BIAS_RESID, OPL_B_KMAJOR)
+#undef TP_GEMM_PICK
+  return nullptr;
+}
+
+static int operand_layout(const GemmArgs& a) { return (a.a_mn ? OPL_A_MN : 0) | (a.b_kmajor ? OPL_B_KMAJOR : 0); }
+
+constexpr int NUM_EPI = 6;
+static int g_pair_clusters[64] = {0};
+static bool g_attr_set[64][2][NUM_EPI][4] = {};
+
+// Allow the kernel's dynamic shared memory (once per device and instantiation).
+static tp_status set_smem_attr(int dev, int epi, int opl, bool pair) {
+  const bool known = dev >= 0 && dev < 64 && epi >= 0 && epi < NUM_EPI && opl >= 0 && opl < 4;
+  if (known && g_attr_set[dev][pair][epi][opl]) return TP_OK;
+  GemmKernel k = gemm_kernel_for(epi, opl, pair);
+  if (!k) return set_error(TP_ERR_CUDA, "no GEMM instantiation for this epilogue and operand layout");
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pair ? P_SMEM_BYTES : SMEM_BYTES) !=
+      cudaSuccess)
+    return set_error(TP_ERR_CUDA, "cudaFuncSetAttribute (shared memory) failed");
+  if (known) g_attr_set[dev][pair][epi][opl] = true;
+  return TP_OK;
+}
+
+// Largest number of co-resident CTA pairs for the pair kernel on this device (every
+// instantiation has the same block size and shared memory).
 static int pair_clusters(int dev) {
   if (dev < 0 || dev >= 64) return 0;
   if (g_pair_clusters[dev]) return g_pair_clusters[dev];
-  if (cudaFuncSetAttribute(tp_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES) !=
-      cudaSuccess)
-    return -1;
+  if (set_smem_attr(dev, EPI_ACT, 0, true) != TP_OK) return -1;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -940,7 +992,7 @@ static int pair_clusters(int dev) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, tp_gemm_pair_kernel, &cfg) != cudaSuccess || n <= 0) return -1;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_kernel_for(EPI_ACT, 0, true), &cfg) != cudaSuccess || n <= 0) return -1;
   g_pair_clusters[dev] = n;
   return n;
 }
@@ -948,36 +1000,36 @@ static int pair_clusters(int dev) {
 static tp_status launch_gemm_pair(const GemmArgs& a, cudaStream_t stream, const char* name, int dev) {
   const int nclusters_max = pair_clusters(dev);
   if (nclusters_max <= 0) return TP_ERR_CUDA;
+  const int opl = operand_layout(a);
+  const tp_status sa = set_smem_attr(dev, a.epi, opl, true);
+  if (sa != TP_OK) return sa;
   const int m_tiles = (a.M + P_ROWS - 1) / P_ROWS;
   const int n_tiles = (a.N + BN - 1) / BN;
   const long long tiles = 1LL * m_tiles * n_tiles * (a.concat ? 1 : a.G);
   if (tiles <= 0) return TP_OK;
   const int nclusters = static_cast<int>(tiles < nclusters_max ? tiles : nclusters_max);
   trace_before(stream);
-  const tp_status st = launch_ex(tp_gemm_pair_kernel, dim3(2 * nclusters), dim3(THREADS), P_SMEM_BYTES, stream, 2, a);
+  const tp_status st = launch_ex(gemm_kernel_for(a.epi, opl, true), dim3(2 * nclusters), dim3(THREADS), P_SMEM_BYTES,
+                                 stream, 2, a);
   if (st != TP_OK) return st;
   trace_after(stream, name);
   return TP_OK;
 }
 
 tp_status launch_gemm(const GemmArgs& a, cudaStream_t stream, const char* name) {
-  static int attr_set[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return TP_ERR_CUDA;
   if (gemm_use_pairs()) return launch_gemm_pair(a, stream, name, dev);
-  if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(tp_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
-        cudaSuccess)
-      return TP_ERR_CUDA;
-    attr_set[dev] = 1;
-  }
+  const int opl = operand_layout(a);
+  const tp_status sa = set_smem_attr(dev, a.epi, opl, false);
+  if (sa != TP_OK) return sa;
   const int m_tiles = (a.M + BM - 1) / BM;
   const int n_tiles = (a.N + BN - 1) / BN;
   const long long tiles = 1LL * m_tiles * n_tiles * (a.concat ? 1 : a.G);
   if (tiles <= 0) return TP_OK;
   const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
   trace_before(stream);
-  const tp_status st = launch_ex(tp_gemm_kernel, dim3(grid), dim3(THREADS), SMEM_BYTES, stream, 1, a);
+  const tp_status st = launch_ex(gemm_kernel_for(a.epi, opl, false), dim3(grid), dim3(THREADS), SMEM_BYTES, stream, 1, a);
   if (st != TP_OK) return st;
   trace_after(stream, name);
   return TP_OK;
