@@ -185,6 +185,24 @@ tp_status make_tmap_out(CUtensorMap* map, void* base, int f16, uint64_t cols, ui
   return TP_OK;
 }
 
+// fp32 output map of a grouped GEMM: (cols, rows, groups) with the given row and group
+// strides, box {16 columns, 32 rows, 1 group}, 64-byte swizzle: a tile's stores clip at its
+// own group's edge.
+tp_status make_tmap_out_f32_3d(CUtensorMap* map, void* base, uint64_t cols, uint64_t rows, uint64_t groups,
+                               uint64_t row_stride_bytes, uint64_t group_stride_bytes) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[3] = {cols, rows, groups};
+  cuuint64_t strides[2] = {row_stride_bytes, group_stride_bytes};
+  cuuint32_t box[3] = {16, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled(out f32) failed (%d)", static_cast<int>(r));
+  return TP_OK;
+}
+
 static tp_status make_tmap_f16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                                    uint64_t s1_bytes, uint64_t s2_bytes, uint32_t b0, uint32_t b1) {
   EncodeTiledFn enc = encode_fn();
@@ -356,6 +374,8 @@ tp_status run_row(const void* A, int64_t M, int64_t kg, int64_t n, int t, const 
   a.epi = EPI_PARTIAL_F32;
   a.out = P; a.ld_out = n; a.out_group_stride = M * n;
   if (separate_reduce()) {
+    TP_TRY(make_tmap_out_f32_3d(&a.tmOut, P, n, M, t, n * 4, M * n * 4));
+    a.tma_store = 1;
     TP_TRY(launch_gemm(a, stream, "gemm_row_partials"));
     return launch_reduce_partials(P, t, M, n, bias, 0, resid, resid_fp32, out, out_fp32, stream);
   }
@@ -363,7 +383,9 @@ tp_status run_row(const void* A, int64_t M, int64_t kg, int64_t n, int t, const 
   // one is added to them straight from the accumulator, in the order 0..t-1
   a.counters = row_partials_counters(P, M, n, t);
   a.red_out = out; a.red_out_f32 = out_fp32;
-  if (!out_fp32) TP_TRY(make_tmap_out(&a.tmOut, out, 0, static_cast<uint64_t>(n), M, n * 2));
+  TP_TRY(make_tmap_out_f32_3d(&a.tmOut, P, n, M, t, n * 4, M * n * 4));
+  a.tma_store = 1;
+  if (!out_fp32) TP_TRY(make_tmap_out(&a.tmOut2, out, 0, static_cast<uint64_t>(n), M, n * 2));
   a.bias = bias; a.resid = resid; a.ld_resid = n; a.resid_fp32 = resid_fp32;
   return launch_gemm(a, stream, "gemm_row_partials");
 }
@@ -481,6 +503,8 @@ tp_status ffn_backward_bf16(const void* X, int64_t M, int64_t h, int64_t f, int 
     a.a_mn = 1; a.a_m_per_group = static_cast<int>(fs);
     a.epi = EPI_PARTIAL_F32;
     a.out = dW2; a.ld_out = h; a.out_group_stride = fs * h;
+    TP_TRY(make_tmap_out_f32_3d(&a.tmOut, dW2, h, fs, t, h * 4, fs * h * 4));
+    a.tma_store = 1;
     a.status = status; a.wait_limit_ns = lim;
     TP_TRY(launch_gemm(a, stream, "gemm_bwd_dw2"));
   }
@@ -494,6 +518,8 @@ tp_status ffn_backward_bf16(const void* X, int64_t M, int64_t h, int64_t f, int 
     a.a_mn = 1; a.a_m_per_group = 0;
     a.epi = EPI_PARTIAL_F32;
     a.out = dW1; a.ld_out = f; a.out_group_stride = fs;
+    TP_TRY(make_tmap_out_f32_3d(&a.tmOut, dW1, fs, h, t, f * 4, fs * 4));
+    a.tma_store = 1;
     a.status = status; a.wait_limit_ns = lim;
     TP_TRY(launch_gemm(a, stream, "gemm_bwd_dw1"));
   }

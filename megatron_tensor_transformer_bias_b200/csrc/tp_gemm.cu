@@ -157,22 +157,15 @@ __device__ __forceinline__ void epilogue_math(const GemmArgs& a, const TileCoord
 // position j ^ ((r >> 1) & 3) of its 64-byte row (no bank conflicts).  Lane 0
 // stores the chunk at (x, y0) and recycles a buffer once the store issued two
 // chunks earlier has read it.
-__device__ __forceinline__ void stage_and_store(const GemmArgs& a, const CUtensorMap* map, int out_type,
-                                                uint8_t* warp_staging, int& count, int lane, const float (&v)[32],
-                                                int x, int y0) {
+// Stage 16 32-bit words per lane (a 32-row x 64-byte box) and store the box with TMA:
+// 2-D at (x, y0), or 3-D at (x, y0, z) when z >= 0.
+__device__ __forceinline__ void stage_words_and_store(const GemmArgs& a, const CUtensorMap* map,
+                                                      uint8_t* warp_staging, int& count, int lane,
+                                                      const uint32_t (&pk)[16], int x, int y0, int z) {
   uint8_t* buf = warp_staging + (count & 1) * 2048;
   if (count >= 2) {
     if (lane == 0) bulk_wait_group_read<1>();
     __syncwarp();
-  }
-  uint32_t pk[16];
-  if (out_type == OUT_F16) {
-    note_f16_range(a.status, absmax32(v), DEV_RANGE_COLUMN);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) pk[i] = pack_f16x2(v[2 * i], v[2 * i + 1]);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
   }
   const int sw = (lane >> 1) & 3;
 #pragma unroll
@@ -182,10 +175,28 @@ __device__ __forceinline__ void stage_and_store(const GemmArgs& a, const CUtenso
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0 && y0 < a.M) {
-    tma_store_2d(map, buf, x, y0);
+    if (z < 0)
+      tma_store_2d(map, buf, x, y0);
+    else
+      tma_store_3d(map, buf, x, y0, z);
     bulk_commit_group();
   }
   ++count;
+}
+
+__device__ __forceinline__ void stage_and_store(const GemmArgs& a, const CUtensorMap* map, int out_type,
+                                                uint8_t* warp_staging, int& count, int lane, const float (&v)[32],
+                                                int x, int y0) {
+  uint32_t pk[16];
+  if (out_type == OUT_F16) {
+    note_f16_range(a.status, absmax32(v), DEV_RANGE_COLUMN);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) pk[i] = pack_f16x2(v[2 * i], v[2 * i + 1]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+  }
+  stage_words_and_store(a, map, warp_staging, count, lane, pk, x, y0, -1);
 }
 
 __device__ __forceinline__ void load_f16x32(const void* p, float (&v)[32]) {
@@ -224,6 +235,17 @@ __device__ __forceinline__ void epilogue_tma_chunk(const GemmArgs& a, const Tile
     stage_and_store(a, &a.tmOut2, OUT_F16, warp_staging, count, lane, gr, x, y0);
     return;
   }
+  if (EPI == EPI_PARTIAL_F32) {
+    // fp32 output through a 3-D map (column, row, group): two 16-column boxes per chunk
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) pk[i] = __float_as_uint(v[half * 16 + i]);
+      stage_words_and_store(a, &a.tmOut, warp_staging, count, lane, pk, n + half * 16, y0, tc.g);
+    }
+    return;
+  }
   if (EPI == EPI_MUL_GRAD) {
     // dZ = dA * act'(Z): the factor sits at the output's own position
     if (row < a.M) {
@@ -251,7 +273,7 @@ __device__ __forceinline__ void load_f32x32_cg(const float* p, float (&v)[32]) {
 // Step 3 inside the row GEMM (partials mode, a.red_out set).  Tiles run in the order
 // m, n, group, so in every CTA pair's sequence all tiles of groups 0..G-2 come before any
 // tile of group G-1.  A warp of a group g < G-1 tile stores its 32-row x 128-column region
-// of the fp32 partial P_g and counts it on the region's arrival counter.  The warp of the
+// of the fp32 partial P_g (TMA stores) and counts it on the region's arrival counter.  The warp of the
 // group G-1 tile that covers the same region waits (bounded) until the G-1 earlier
 // partials are counted -- they were stored before their pairs started any group G-1
 // tile, so the wait always ends -- and then sums P_0 .. P_{G-2} from memory and its own
@@ -264,12 +286,18 @@ __device__ __forceinline__ int region_counter(const GemmArgs& a, int row0, int c
   return (row0 / 32) * ((a.N + 127) / 128) + col_region;
 }
 
-// Publish this warp's stores of its region of a partial: each lane's stores are fenced
-// before lane 0's atomic.
+// Publish this warp's region of a partial.  Its lane 0 issued the region's TMA stores: it
+// waits for them to complete, orders them before its generic accesses, and fences before the
+// atomic that counts the region.
 __device__ __forceinline__ void partial_signal(const GemmArgs& a, int ctr, int lane) {
-  __threadfence();
   __syncwarp();
-  if (lane == 0) atomicAdd(&a.counters[ctr], 1u);
+  if (lane == 0) {
+    bulk_wait_group_all();
+    fence_proxy_async_global();
+    __threadfence();
+    atomicAdd(&a.counters[ctr], 1u);
+  }
+  __syncwarp();
 }
 
 // Wait until the region's G-1 earlier partials are counted; fenced so that the warp's
@@ -298,7 +326,7 @@ __device__ __forceinline__ bool partial_wait(const GemmArgs& a, int ctr, int lan
 }
 
 // One 32-column chunk of a group G-1 tile: out = ((P_0 + P_1) + ...) + P_{G-1} + bias + resid,
-// taken 16 columns at a time (the result replaces v) to keep the registers in check.  The
+// taken 8 columns at a time (the result replaces v) to keep the registers in check.  The
 // partials were written earlier in this launch: they are read with plain (L1-allocating)
 // loads, never through the read-only path, and no line of them was in this SM's L1 before.
 __device__ __forceinline__ void reduce_chunk(const GemmArgs& a, int row, int n, float (&v)[32], bool ok,
@@ -306,31 +334,43 @@ __device__ __forceinline__ void reduce_chunk(const GemmArgs& a, int row, int n, 
   if (row < a.M && ok) {
     const float* p = static_cast<const float*>(a.out) + static_cast<int64_t>(row) * a.ld_out + n;
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      float acc[16];
-      if (a.G > 1) {
-        const float4* q0 = reinterpret_cast<const float4*>(p + half * 16);
+    for (int qt = 0; qt < 4; ++qt) {
+      float4 acc[2];
+      // 8 columns at a time: the loads of partials 0..G-2 (up to four at a time) are all
+      // issued before the adds, which then run in the order 0, 1, 2, ...
+      for (int g0 = 0; g0 < a.G - 1; g0 += 4) {
+        float4 w[4][2];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float4 u = q0[i];
-          acc[i * 4] = u.x; acc[i * 4 + 1] = u.y; acc[i * 4 + 2] = u.z; acc[i * 4 + 3] = u.w;
-        }
-        for (int g = 1; g < a.G - 1; ++g) {
-          const float4* q = reinterpret_cast<const float4*>(p + static_cast<int64_t>(g) * a.out_group_stride + half * 16);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float4 u = q[i];
-            acc[i * 4] += u.x; acc[i * 4 + 1] += u.y; acc[i * 4 + 2] += u.z; acc[i * 4 + 3] += u.w;
+        for (int u = 0; u < 4; ++u) {
+          if (g0 + u < a.G - 1) {
+            const float4* q =
+                reinterpret_cast<const float4*>(p + static_cast<int64_t>(g0 + u) * a.out_group_stride + qt * 8);
+            w[u][0] = q[0];
+            w[u][1] = q[1];
           }
         }
 #pragma unroll
-        for (int j = 0; j < 16; ++j) acc[j] += v[half * 16 + j];
-      } else {
+        for (int u = 0; u < 4; ++u) {
+          if (g0 + u < a.G - 1) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) acc[j] = v[half * 16 + j];
+            for (int i = 0; i < 2; ++i) {
+              if (g0 + u == 0) {
+                acc[i] = w[u][i];
+              } else {
+                acc[i].x += w[u][i].x; acc[i].y += w[u][i].y; acc[i].z += w[u][i].z; acc[i].w += w[u][i].w;
+              }
+            }
+          }
+        }
       }
+      // then the last partial, straight from the accumulator
+      if (a.G > 1) {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) v[half * 16 + j] = acc[j];
+        for (int i = 0; i < 2; ++i) {
+          float* d = &v[qt * 8 + i * 4];
+          d[0] = acc[i].x + d[0]; d[1] = acc[i].y + d[1]; d[2] = acc[i].z + d[2]; d[3] = acc[i].w + d[3];
+        }
+      }
     }
     if (a.bias) {
       float b[32];
@@ -351,7 +391,7 @@ __device__ __forceinline__ void reduce_chunk(const GemmArgs& a, int row, int n, 
   if (a.red_out_f32) {
     if (row < a.M) store_f32x32(static_cast<float*>(a.red_out) + static_cast<int64_t>(row) * a.N + n, v);
   } else {
-    stage_and_store(a, &a.tmOut, OUT_BF16, warp_staging, count, lane, v, n, row - lane);
+    stage_and_store(a, &a.tmOut2, OUT_BF16, warp_staging, count, lane, v, n, row - lane);
   }
 }
 
@@ -476,7 +516,8 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_base_slot;
-  pdl_wait();  // the previous kernel's outputs (our operands, our workspace) are complete
+  // Dependents may start once every CTA of this grid is resident (see the pair kernel).
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -487,6 +528,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
       // both operands are re-read by several CTAs at about the same time: default L2 policy
       const uint64_t pol_a = l2_policy_evict_normal();
       const uint64_t pol_b = pol_a;
+      pdl_wait();  // the previous kernel's outputs (our operands) are complete
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
@@ -586,9 +628,10 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
     int acc = 0;
     uint32_t acc_phase = 0;
     const bool tma_out = a.tma_store && (EPI == EPI_ACT || EPI == EPI_BIAS_RESID || EPI == EPI_ACT_GRAD ||
-                                         EPI == EPI_MUL_GRAD);
+                                         EPI == EPI_MUL_GRAD || EPI == EPI_PARTIAL_F32);
     uint8_t* warp_staging = staging + (warp - 2) * 4096;
     int store_count = 0;
+    pdl_wait();  // bias / residual inputs and our outputs: after the previous kernel completes
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       if (*abort_flag) break;
       // the decision is made warp-uniform: tcgen05.ld below is a warp-collective instruction
@@ -619,7 +662,18 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
         red_ok = partial_wait(a, ctr, lane);
         if (!red_ok) *abort_flag = 1;
       }
-      if (c_begin < c_end) {
+      if (c_begin < c_end && red_tile) {
+        // last shard's tile: one chunk at a time (the registers go to the partials' loads)
+        for (int c = c_begin; c < c_end; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_row + c * 32, r);
+          tmem_ld_wait();
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          reduce_chunk(a, row, n0 + c * 32, v, red_ok, warp_staging, store_count, lane);
+        }
+      } else if (c_begin < c_end) {
         uint32_t r[2][32];
         tmem_ld_32x32b_x32(t_row + c_begin * 32, r[0]);
 #pragma unroll
@@ -631,9 +685,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
           float v[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[cur][j]);
-          if (red_tile) {
-            reduce_chunk(a, row, n0 + c * 32, v, red_ok, warp_staging, store_count, lane);
-          } else if (tma_out) {
+          if (tma_out) {
             const int x = (EPI == EPI_BIAS_RESID ? 0 : tc.g * static_cast<int>(a.out_col_per_group)) + n0 + c * 32;
             epilogue_tma_chunk<EPI>(a, tc, row, n0 + c * 32, v, warp_staging, store_count, lane, x, row - lane);
           } else if (row < a.M) {
@@ -651,7 +703,6 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
     if (lane == 0) bulk_wait_group_all();  // our output stores are complete before exit
   }
 
-  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -730,7 +781,10 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
   cluster_sync_all();  // barriers of both CTAs initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_base_slot;
-  pdl_wait();  // the previous kernel's outputs (our operands, our workspace) are complete
+  // The next kernel may be scheduled onto SMs this grid leaves idle in its tail.  It starts
+  // only once every CTA of this grid has issued this, i.e. is resident, so it cannot take
+  // an SM this grid still needs; its own wait keeps it from our outputs until we finish.
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -742,6 +796,26 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
       const uint64_t pol_a = l2_policy_evict_normal();
       const uint64_t pol_b = pol_a;
       const uint32_t full0_leader = mapa_shared(smem_u32(&full_bar[0]), 0);
+      // Before waiting for the previous kernel: pull the first stages of this CTA's first
+      // tile into L2 (prefetch only; the loads into shared memory come after the wait).
+      if (cid < num_tiles) {
+        const TileCoord tc = tile_coord(a, cid, m_tiles, n_tiles);
+        const int m0 = tc.m_blk * P_ROWS + static_cast<int>(rank) * BM;
+        const int n0 = tc.n_blk * BN + static_cast<int>(rank) * (BN / 2);
+        const bool rev = a.concat != 0;
+        const int pre = k_iters < P_STAGES ? k_iters : P_STAGES;
+        for (int it = 0; it < pre; ++it) {
+          const int kidx = rev ? k_iters - 1 - it : it;
+          const int g = a.concat ? kidx / kb_per_group : tc.g;
+          const int kb = a.concat ? kidx - g * kb_per_group : kidx;
+          const int ka = g * a.a_k_per_group + kb * BK;
+          if (!A_MN) tma_prefetch_l2_2d(&a.tmA, ka, m0);
+          else tma_prefetch_l2_3d(&a.tmA, 0, ka, (g * a.a_m_per_group + m0) / 64);
+          if (!B_KM) tma_prefetch_l2_3d(&a.tmB[g], 0, kb * BK, n0 / 64);
+          else tma_prefetch_l2_2d(&a.tmB[g], kb * BK, n0);
+        }
+      }
+      pdl_wait();  // the previous kernel's outputs (our operands) are complete
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
@@ -842,10 +916,11 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
     const int row_in_tile = static_cast<int>(rank) * BM + sub * 32 + lane;
     const int col_half = (warp - 2) / 4;    // columns [col_half*BN/2, +BN/2) of each tile
     const uint32_t acc_empty0_leader = mapa_shared(smem_u32(&acc_empty[0]), 0);
+    pdl_wait();  // bias / residual inputs and our outputs: after the previous kernel completes
     int acc = 0;
     uint32_t acc_phase = 0;
     const bool tma_out = a.tma_store && (EPI == EPI_ACT || EPI == EPI_BIAS_RESID || EPI == EPI_ACT_GRAD ||
-                                         EPI == EPI_MUL_GRAD);
+                                         EPI == EPI_MUL_GRAD || EPI == EPI_PARTIAL_F32);
     uint8_t* warp_staging = staging + (warp - 2) * 4096;
     int store_count = 0;
     for (int tile = cid; tile < num_tiles; tile += nclusters) {
@@ -877,7 +952,18 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
         red_ok = partial_wait(a, ctr, lane);
         if (!red_ok) *abort_flag = 1;
       }
-      if (c_begin < c_end) {
+      if (c_begin < c_end && red_tile) {
+        // last shard's tile: one chunk at a time (the registers go to the partials' loads)
+        for (int c = c_begin; c < c_end; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_row + c * 32, r);
+          tmem_ld_wait();
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          reduce_chunk(a, row, n0 + c * 32, v, red_ok, warp_staging, store_count, lane);
+        }
+      } else if (c_begin < c_end) {
         uint32_t r[2][32];
         tmem_ld_32x32b_x32(t_row + c_begin * 32, r[0]);
 #pragma unroll
@@ -889,9 +975,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
           float v[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[cur][j]);
-          if (red_tile) {
-            reduce_chunk(a, row, n0 + c * 32, v, red_ok, warp_staging, store_count, lane);
-          } else if (tma_out) {
+          if (tma_out) {
             const int x = (EPI == EPI_BIAS_RESID ? 0 : tc.g * static_cast<int>(a.out_col_per_group)) + n0 + c * 32;
             epilogue_tma_chunk<EPI>(a, tc, row, n0 + c * 32, v, warp_staging, store_count, lane, x, row - lane);
           } else if (row < a.M) {
@@ -909,7 +993,6 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
     if (lane == 0) bulk_wait_group_all();  // our output stores are complete before exit
   }
 
-  pdl_launch_dependents();
   __syncwarp();
   tc_fence_before();
   cluster_sync_all();  // the leader's MMAs and the remote arrives are done in both CTAs

@@ -48,8 +48,12 @@ enum OutType : int { OUT_BF16 = 0, OUT_F32 = 1, OUT_F16 = 2 };
 enum Activation : int { ACT_NONE = 0, ACT_GELU = 1, ACT_RELU = 2 };
 
 struct __align__(64) GemmArgs {
-  CUtensorMap tmOut;                    // 16-bit output of the TMA-store epilogues, box {32, 32}, 64B swizzle
-  CUtensorMap tmOut2;                   // EPI_ACT_GRAD: act'(z) output (fp16), same box
+  // Output of the TMA-store epilogues: 16-bit [rows, cols], box {32, 32}; or, for
+  // EPI_PARTIAL_F32, fp32 (cols, rows, group), box {16, 32, 1}.  64B swizzle.
+  CUtensorMap tmOut;
+  // EPI_ACT_GRAD: act'(z) output (fp16); partials mode with the in-GEMM reduction: the bf16
+  // output [M, N].  Box {32, 32}, 64B swizzle.
+  CUtensorMap tmOut2;
   // A [M, Ktot] K-major: box {64 K, 128 M}; or (a_mn) the matrix [Ktot, M] with M
   // contiguous: a make_tmap_mn map (box {64 M, 64 K, 2 blocks}).  128B swizzle.
   CUtensorMap tmA;
