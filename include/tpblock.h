@@ -81,14 +81,13 @@ typedef enum { TP_BF16 = 0, TP_FP32 = 1, TP_FP16 = 2 } tp_dtype;
  *                     B200), so the bits are reproducible across runs and
  *                     processes on devices with the same SM count.
  * TP_REDUCE_PARTIALS: the row GEMM writes t fp32 partials Y_i [t, M, h] to the
- *                     workspace.  Inside the same kernel, the shard that is the
- *                     last to finish a 32-row x 128-column region of the
- *                     output sums that region's t partials in the order
- *                     0..t-1 and adds bias and residual, so the reduction
- *                     runs while other tiles are still being multiplied
- *                     ([TP-CR] step 3 overlapped with step 2).  The sums are
- *                     the ones a separate pass over the partials would take:
- *                     same order, same bits. */
+ *                     workspace (TMA stores) and a reduce kernel sums them in
+ *                     the order 0..t-1, then adds bias and residual.  With the
+ *                     environment variable TPB_REDUCE_IN_GEMM=1 the sum is
+ *                     taken inside the row GEMM instead: its last shard's
+ *                     tiles add the stored partials 0..t-2 and their own
+ *                     accumulator in the same order (same bits), overlapping
+ *                     the reduction with the other tiles' multiplication. */
 typedef enum { TP_REDUCE_FUSED = 0, TP_REDUCE_PARTIALS = 1 } tp_reduce_mode;
 
 /* Element-wise nonlinearity of step 1: exact GeLU z*Phi(z) (erf form) or ReLU. */
@@ -127,9 +126,9 @@ typedef void* tp_stream_t; /* cudaStream_t */
  *  mode     see tp_reduce_mode (ignored for TP_FP32, which always uses partials).
  *  ws       device workspace of at least tp_ffn_workspace_bytes(...) bytes,
  *           256-byte aligned.  Holds act(Z) [M, f] (and, in TP_REDUCE_PARTIALS
- *           mode, the partials and one arrival counter per 32x128 output region,
- *           which the call zeroes on the stream first).  Its contents on entry
- *           are ignored.
+ *           mode, the partials and one arrival counter per 32x128 output region
+ *           for the in-GEMM reduction, which the call zeroes on the stream
+ *           first).  Its contents on entry are ignored.
  * Limits: 1 <= t <= TP_MAX_SHARDS, f % t == 0, M >= 1.
  */
 TP_API size_t tp_ffn_workspace_bytes(int64_t M, int64_t h, int64_t f, int t, tp_dtype dtype, tp_reduce_mode mode);

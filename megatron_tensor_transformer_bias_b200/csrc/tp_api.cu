@@ -283,13 +283,16 @@ uint32_t* row_partials_counters(float* P, int64_t M, int64_t n, int t) {
   return reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(P) + align_up(static_cast<size_t>(t) * M * n * 4));
 }
 
-// The separate reduce kernel instead of the reduction in the row GEMM's epilogue
-// (TPB_SEPARATE_REDUCE=1; the same sums in the same order).
+// Partials mode sums the t partials with the fixed-order reduce kernel after the row GEMM.
+// TPB_REDUCE_IN_GEMM=1 takes the sum inside the row GEMM instead (the last shard's tiles add
+// the stored partials 0..t-2 and their own; same order, same bits).  On one B200 the in-GEMM
+// form is the slower one: the t-1 stored partials come back from DRAM in the last 1/t of
+// the launch, when the row tiles of every region finish at once.
 bool separate_reduce() {
   static int v = -1;
   if (v < 0) {
-    const char* e = getenv("TPB_SEPARATE_REDUCE");
-    v = (e && e[0] == '1') ? 1 : 0;
+    const char* e = getenv("TPB_REDUCE_IN_GEMM");
+    v = (e && e[0] == '1') ? 0 : 1;
   }
   return v == 1;
 }

@@ -1,5 +1,7 @@
 """GPU unit tests of the building blocks: LayerNorm, the fixed-order reduce, the
 bounded-wait status path and the launch trace."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -81,8 +83,12 @@ def test_launch_trace_names_kernels():
     finally:
         tb.tp_trace_disable()
     names = [n for n, _ in recs]
-    # partials mode: the last shard's tiles sum the partials inside the row GEMM
-    assert names == ["gemm_column_act", "gemm_row_partials"]
+    # partials mode: the fixed-order reduce runs after the row GEMM (inside it with
+    # TPB_REDUCE_IN_GEMM=1)
+    if os.environ.get("TPB_REDUCE_IN_GEMM") == "1":
+        assert names == ["gemm_column_act", "gemm_row_partials"]
+    else:
+        assert names == ["gemm_column_act", "gemm_row_partials", "reduce_partials"]
     assert all(ms > 0 for _, ms in recs)
 
 

@@ -165,12 +165,12 @@ def _row_partials_case(M, n, t):
 
 
 def test_row_partials_reduce_matches_separate_pass(tmp_path):
-    """Partials mode sums each region's t partials inside the row GEMM (the last shard's
-    tiles add the stored partials 0..t-2 and their own, in order 0..t-1).  The output must
-    be the same bits as summing the stored partials in a separate pass afterwards, which a
-    child process runs with TPB_SEPARATE_REDUCE=1 on the same inputs; the partials 0..t-2
-    left in the workspace must match too, and two calls in a row must agree (the arrival
-    counters start from zero every call)."""
+    """Partials mode sums the stored partials in a separate fixed-order pass; with
+    TPB_REDUCE_IN_GEMM=1 (run here in a child process on the same inputs) the last shard's
+    tiles add the stored partials 0..t-2 and their own inside the row GEMM, in the order
+    0..t-1.  Both outputs must be the same bits, the partials 0..t-2 left in the workspace
+    too, and two calls in a row must agree (the arrival counters start from zero every
+    call)."""
     import subprocess
     import sys
     here = {}
@@ -182,7 +182,7 @@ def test_row_partials_reduce_matches_separate_pass(tmp_path):
     code = ("import sys, torch; sys.path.insert(0, %r); from tests import test_gpu_ffn as T; "
             "torch.save({c: tuple(x.cpu() for x in (T._row_partials_case(*c)[0][0], T._row_partials_case(*c)[1])) "
             "for c in T.ROW_PARTIAL_CASES}, %r)" % (ROOT, str(dump)))
-    r = subprocess.run([sys.executable, "-c", code], env=dict(os.environ, TPB_SEPARATE_REDUCE="1"),
+    r = subprocess.run([sys.executable, "-c", code], env=dict(os.environ, TPB_REDUCE_IN_GEMM="1"),
                        capture_output=True, text=True, timeout=600, cwd=ROOT)
     assert r.returncode == 0, r.stderr[-3000:]
     there = torch.load(dump)

@@ -1,7 +1,7 @@
 """The library's launch switches, read once per process from the environment:
 TPB_GEMM_PAIRS=0 runs every GEMM on the one-CTA kernel (128x256 tiles) instead of CTA
-pairs, TPB_PDL=0 launches without programmatic dependent launch, TPB_SEPARATE_REDUCE=1
-sums the partials in a separate kernel after the row GEMM instead of in its epilogue.  Each is exercised by
+pairs, TPB_PDL=0 launches without programmatic dependent launch, TPB_REDUCE_IN_GEMM=1
+sums the partials inside the row GEMM instead of in a separate kernel after it.  Each is exercised by
 re-running small parity tests against the oracle in a child process."""
 import os
 import subprocess
@@ -23,11 +23,12 @@ CASES = [
     "tests/test_gpu_attention_layer.py::test_attention_small_full",
     "tests/test_gpu_attention_layer.py::test_layer_small_full",
     "tests/test_gpu_backward.py::test_backward_small_full",
+    "tests/test_gpu_blocks.py::test_launch_trace_names_kernels",
 ]
 
 
-@pytest.mark.parametrize("env", [{"TPB_GEMM_PAIRS": "0"}, {"TPB_PDL": "0"}, {"TPB_SEPARATE_REDUCE": "1"}],
-                         ids=["one_cta_gemm", "no_pdl", "separate_reduce_kernel"])
+@pytest.mark.parametrize("env", [{"TPB_GEMM_PAIRS": "0"}, {"TPB_PDL": "0"}, {"TPB_REDUCE_IN_GEMM": "1"}],
+                         ids=["one_cta_gemm", "no_pdl", "reduce_in_gemm"])
 def test_parity_under_switch(env):
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider", *CASES],
                        cwd=ROOT, env=dict(os.environ, **env), capture_output=True, text=True, timeout=900)
