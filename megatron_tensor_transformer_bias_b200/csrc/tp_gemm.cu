@@ -135,20 +135,23 @@ __device__ __forceinline__ void epilogue_math(const GemmArgs& a, const TileCoord
   if (bias) {
     float b[32];
     load_bf16x32(static_cast<const uint16_t*>(bias) + n, b);
-#pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] += b[j];
+    add32(v, b);
   }
   if (EPI == EPI_ACT) {
+    if (a.act == ACT_GELU) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = act_apply(v[j], a.act);
+      for (int j = 0; j < 32; j += 2) gelu_exact2(v[j], v[j + 1]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = act_apply(v[j], a.act);
+    }
   } else if (a.resid && row < a.M) {
     float r[32];
     if (a.resid_fp32)
       load_f32x32(static_cast<const float*>(a.resid) + static_cast<int64_t>(row) * a.ld_resid + n, r);
     else
       load_bf16x32(static_cast<const uint16_t*>(a.resid) + static_cast<int64_t>(row) * a.ld_resid + n, r);
-#pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] += r[j];
+    add32(v, r);
   }
 }
 

@@ -429,6 +429,67 @@ __device__ __forceinline__ float gelu_exact(float x) {
   return x * (x >= 0.0f ? 1.0f - half_erfc : half_erfc);
 }
 
+// ---------------------------------------------------------------- packed fp32x2 arithmetic
+// Two IEEE fp32 operations in one instruction: each lane of fma.rn.f32x2 / mul.rn.f32x2 is
+// exactly the scalar fmaf / __fmul_rn, so code written with them gives the same bits.
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                     float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void mul2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// v[j] += w[j] for 32 values, two at a time (same bits as the scalar adds).
+__device__ __forceinline__ void add32(float (&v)[32], const float (&w)[32]) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) add2(v[j], v[j + 1], v[j], v[j + 1], w[j], w[j + 1]);
+}
+
+// gelu_exact on two values at once, with the same operations in the same order (same bits).
+__device__ __forceinline__ void gelu_exact2(float& x0, float& x1) {
+  float z0, z1;
+  mul2(z0, z1, fabsf(x0), fabsf(x1), 0.70710678118654752f, 0.70710678118654752f);
+  float d0, d1;
+  fma2(d0, d1, 0.5f, 0.5f, z0, z1, 1.0f, 1.0f);
+  const float t0 = __fdividef(1.0f, d0), t1 = __fdividef(1.0f, d1);
+  float p0 = 0.17087277f, p1 = 0.17087277f;
+  fma2(p0, p1, p0, p1, t0, t1, -0.82215223f, -0.82215223f);
+  fma2(p0, p1, p0, p1, t0, t1, 1.48851587f, 1.48851587f);
+  fma2(p0, p1, p0, p1, t0, t1, -1.13520398f, -1.13520398f);
+  fma2(p0, p1, p0, p1, t0, t1, 0.27886807f, 0.27886807f);
+  fma2(p0, p1, p0, p1, t0, t1, -0.18628806f, -0.18628806f);
+  fma2(p0, p1, p0, p1, t0, t1, 0.09678418f, 0.09678418f);
+  fma2(p0, p1, p0, p1, t0, t1, 0.37409196f, 0.37409196f);
+  fma2(p0, p1, p0, p1, t0, t1, 1.00002368f, 1.00002368f);
+  fma2(p0, p1, p0, p1, t0, t1, -1.26551223f, -1.26551223f);
+  float a0, a1;
+  fma2(a0, a1, -z0, -z1, z0, z1, p0, p1);
+  const float e0 = __expf(a0), e1 = __expf(a1);
+  float h0, h1;
+  mul2(h0, h1, 0.5f, 0.5f, t0, t1);
+  mul2(h0, h1, h0, h1, e0, e1);
+  const float phi0 = x0 >= 0.0f ? 1.0f - h0 : h0;
+  const float phi1 = x1 >= 0.0f ? 1.0f - h1 : h1;
+  mul2(x0, x1, x0, x1, phi0, phi1);
+}
+
 // GeLU and its derivative together: GeLU'(x) = Phi(x) + x phi(x), phi(x) = exp(-x^2/2) / sqrt(2 pi),
 // with Phi from the same erfc formula as gelu_exact (so GeLU here is bit-identical to it).
 __device__ __forceinline__ float gelu_and_grad(float x, float& grad) {
