@@ -83,6 +83,12 @@ KERNEL_SOURCES = {
     "attention": ["tp_attention.cu"] + _SHARED_SOURCES,
     "reduce_partials": ["tp_simt.cu"] + _SHARED_SOURCES,
     "layernorm": ["tp_simt.cu"] + _SHARED_SOURCES,
+    "gemm_bwd_recompute": ["tp_gemm.cu"] + _SHARED_SOURCES,
+    "gemm_bwd_dz": ["tp_gemm.cu"] + _SHARED_SOURCES,
+    "gemm_bwd_dw2": ["tp_gemm.cu"] + _SHARED_SOURCES,
+    "gemm_bwd_dw1": ["tp_gemm.cu"] + _SHARED_SOURCES,
+    "gemm_bwd_dx": ["tp_gemm.cu"] + _SHARED_SOURCES,
+    "colsum": ["tp_simt.cu"] + _SHARED_SOURCES,
 }
 
 
@@ -335,7 +341,9 @@ class FFNBwd(Workload):
         M, h, f, t = w.M, w.h, w.f, w.t
         self.kernel_amount = {k: ("tensor", 2 * M * h * f, "FLOP") for k in
                               ("gemm_bwd_recompute", "gemm_bwd_dz", "gemm_bwd_dw2", "gemm_bwd_dw1", "gemm_bwd_dx")}
-        self.kernel_amount["colsum"] = ("hbm", M * f * 2 + M * h * 2, "B")
+        # Each step traces four colsum launches: a chunk pass and a final pass for db1 (over dZ)
+        # and for db2 (over dY); their bytes, M*f*2 + M*h*2 in all, are spread over the four.
+        self.kernel_amount["colsum"] = ("hbm", (M * f * 2 + M * h * 2) // 4, "B")
 
     def setup(self, dev, rank):
         import torch
