@@ -614,8 +614,8 @@ tp_status attn_bf16(const void* X, int B, int S, int h, int H, int d, int t, con
     AttnArgs a;
     memset(&a, 0, sizeof(a));
     TP_TRY(make_tmap_attn(&a.tmQ, w.q, B * H, S, d, 128));  // 128-query tiles
-    TP_TRY(make_tmap_attn(&a.tmK, w.k, B * H, S, d, 64));   // 64-key blocks
-    TP_TRY(make_tmap_attn(&a.tmV, w.v, B * H, S, d, 64));
+    TP_TRY(make_tmap_attn(&a.tmK, w.k, B * H, S, d, attention_kv_rows()));  // key blocks of the kernel
+    TP_TRY(make_tmap_attn(&a.tmV, w.v, B * H, S, d, attention_kv_rows()));
     a.O = w.o; a.o_f16 = is_f16(Wo);
     a.B = B; a.S = S; a.H = H; a.d = d; a.causal = causal; a.head0 = 0;
     a.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(d));

@@ -134,6 +134,8 @@ tp_status make_tmap_out(CUtensorMap* map, void* base, int f16, uint64_t cols, ui
 // the C-ABI layer has checked every argument before calling them.
 tp_status launch_gemm(const GemmArgs& a, cudaStream_t stream, const char* name);
 tp_status launch_attention(const AttnArgs& a, cudaStream_t stream);
+// Rows of the K and V tensor-map boxes: the key-block size of the attention kernel in use.
+int attention_kv_rows();
 tp_status launch_reduce_partials(const float* P, int t, int64_t M, int64_t h, const void* bias, int bias_fp32,
                                  const void* resid, int resid_fp32, void* out, int out_fp32,
                                  cudaStream_t stream);

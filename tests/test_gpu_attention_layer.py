@@ -32,7 +32,8 @@ def _attn_ref(a, B, S, H, d, causal=True, rows=None, with_bo=True, with_res=True
                                B, S, H, d, causal=causal, rows=rows)
 
 
-SMALL = [(2, 200, 256, 4), (1, 128, 256, 2), (1, 1, 128, 1), (3, 129, 512, 4), (1, 384, 256, 2), (1, 700, 256, 2)]
+SMALL = [(2, 200, 256, 4), (1, 128, 256, 2), (1, 1, 128, 1), (3, 129, 512, 4), (1, 384, 256, 2), (1, 700, 256, 2),
+         (2, 512, 256, 2), (1, 1000, 256, 2)]
 
 
 @pytest.mark.parametrize("B,S,h,H", SMALL)

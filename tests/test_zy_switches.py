@@ -1,7 +1,9 @@
 """The library's launch switches, read once per process from the environment:
 TPB_GEMM_PAIRS=0 runs every GEMM on the one-CTA kernel (128x256 tiles) instead of CTA
 pairs, TPB_PDL=0 launches without programmatic dependent launch, TPB_REDUCE_IN_GEMM=1
-sums the partials inside the row GEMM instead of in a separate kernel after it.  Each is exercised by
+sums the partials inside the row GEMM instead of in a separate kernel after it,
+TPB_ATTN_ONE_TILE=1 runs attention with one 128-query tile per CTA (64-key blocks, two
+CTAs per SM) instead of two tiles per CTA.  Each is exercised by
 re-running small parity tests against the oracle in a child process."""
 import os
 import subprocess
@@ -27,8 +29,9 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("env", [{"TPB_GEMM_PAIRS": "0"}, {"TPB_PDL": "0"}, {"TPB_REDUCE_IN_GEMM": "1"}],
-                         ids=["one_cta_gemm", "no_pdl", "reduce_in_gemm"])
+@pytest.mark.parametrize("env", [{"TPB_GEMM_PAIRS": "0"}, {"TPB_PDL": "0"}, {"TPB_REDUCE_IN_GEMM": "1"},
+                                 {"TPB_ATTN_ONE_TILE": "1"}],
+                         ids=["one_cta_gemm", "no_pdl", "reduce_in_gemm", "attn_one_tile"])
 def test_parity_under_switch(env):
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider", *CASES],
                        cwd=ROOT, env=dict(os.environ, **env), capture_output=True, text=True, timeout=900)
