@@ -10,6 +10,8 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "tp_internal.h"
 
 namespace tpb {
@@ -105,13 +107,23 @@ tp_status set_error(tp_status s, const char* msg) {
   return s;
 }
 
-void trace_before(cudaStream_t stream) {
+// Every launch is also an NVTX range named after the kernel (start/end ranges, so an
+// error return between the two cannot unbalance a stack); a profiler that records NVTX
+// shows them on the host timeline, without one the calls do nothing.
+thread_local nvtxRangeId_t t_nvtx_launch = 0;
+
+void trace_before(cudaStream_t stream, const char* name) {
+  t_nvtx_launch = nvtxRangeStartA(name);
   if (!t_trace_on || static_cast<int>(t_trace.size()) >= t_trace_cap) return;
   t_pending_start = pool_event(2 * t_trace.size());
   if (t_pending_start) cudaEventRecord(t_pending_start, stream);
 }
 
 void trace_after(cudaStream_t stream, const char* name) {
+  if (t_nvtx_launch) {
+    nvtxRangeEnd(t_nvtx_launch);
+    t_nvtx_launch = 0;
+  }
   if (!t_trace_on || !t_pending_start || static_cast<int>(t_trace.size()) >= t_trace_cap) return;
   cudaEvent_t stop = pool_event(2 * t_trace.size() + 1);
   if (!stop) return;
@@ -650,6 +662,14 @@ tp_status validate_attn(const void* X, int B, int S, int h, int H, int d, int t,
 }  // namespace
 
 // ================================================================ public C ABI
+// NVTX range around one public call (pushed on entry, popped on every return).
+struct ApiRange {
+  explicit ApiRange(const char* name) { nvtxRangePushA(name); }
+  ~ApiRange() { nvtxRangePop(); }
+  ApiRange(const ApiRange&) = delete;
+  ApiRange& operator=(const ApiRange&) = delete;
+};
+
 extern "C" {
 
 size_t tp_ffn_workspace_bytes(int64_t M, int64_t h, int64_t f, int t, tp_dtype dtype, tp_reduce_mode mode) {
@@ -662,6 +682,7 @@ tp_status tp_ffn_forward_act(const void* X, int64_t M, int64_t h, int64_t f, int
                              const void* const* b1, const tp_shard* W2, const void* b2, const void* residual,
                              void* out, tp_dtype dtype, tp_reduce_mode mode, tp_activation act, void* ws,
                              size_t ws_bytes, tp_stream_t stream) {
+  ApiRange range("tp_ffn_forward_act");
   TP_TRY(validate_ffn(X, M, h, f, t, W1, b1, W2, b2, residual, out, dtype, mode, act, ws, ws_bytes));
   if (M == 0) return TP_OK;
   const int kact = act == TP_ACT_GELU ? ACT_GELU : ACT_RELU;
@@ -684,6 +705,7 @@ tp_status tp_ffn_forward(const void* X, int64_t M, int64_t h, int64_t f, int t, 
 
 tp_status tp_column_linear_forward(const void* X, int64_t M, int64_t k, int64_t n, int t, const tp_shard* W,
                                    const void* const* b, int act, void* out, tp_stream_t stream) {
+  ApiRange range("tp_column_linear_forward");
   if (M < 0 || k <= 0 || n <= 0) return fail(TP_ERR_INVALID_ARG, "sizes must be positive (M>=0)");
   if (t < 1 || t > TP_MAX_SHARDS) return fail(TP_ERR_INVALID_ARG, "t outside [1, %d]", TP_MAX_SHARDS);
   if (n % t) return fail(TP_ERR_INVALID_ARG, "n is not divisible by t");
@@ -707,6 +729,7 @@ size_t tp_row_linear_workspace_bytes(int64_t M, int64_t n, int t, tp_reduce_mode
 tp_status tp_row_linear_forward(const void* A, int64_t M, int64_t k, int64_t n, int t, const tp_shard* W,
                                 const void* bias, const void* residual, void* out, tp_reduce_mode mode, void* ws,
                                 size_t ws_bytes, tp_stream_t stream) {
+  ApiRange range("tp_row_linear_forward");
   if (M < 0 || k <= 0 || n <= 0) return fail(TP_ERR_INVALID_ARG, "sizes must be positive (M>=0)");
   if (t < 1 || t > TP_MAX_SHARDS) return fail(TP_ERR_INVALID_ARG, "t outside [1, %d]", TP_MAX_SHARDS);
   if (k % t) return fail(TP_ERR_INVALID_ARG, "k is not divisible by t");
@@ -737,6 +760,7 @@ tp_status tp_ffn_backward(const void* X, int64_t M, int64_t h, int64_t f, int t,
                           const void* const* b1, const tp_shard* W2, const void* dY, const void* dX_add, void* dX,
                           float* dW1, float* db1, float* dW2, float* db2, tp_activation act, void* ws,
                           size_t ws_bytes, tp_stream_t stream) {
+  ApiRange range("tp_ffn_backward");
   if (act != TP_ACT_GELU && act != TP_ACT_RELU) return fail(TP_ERR_INVALID_ARG, "unknown activation %d", act);
   TP_TRY(validate_ffn_bf16_dims(M, h, f, t));
   // with no rows, X, dY and dX are never touched and may be NULL
@@ -782,6 +806,7 @@ tp_status tp_attn_forward(const void* X, int B, int S, int h, int heads, int d, 
                           const void* const* bqkv, const tp_shard* Wo, const void* bo, const void* residual,
                           int causal, void* out, tp_reduce_mode mode, void* ws, size_t ws_bytes,
                           tp_stream_t stream) {
+  ApiRange range("tp_attn_forward");
   if (1LL * B * S == 0) {
     TP_TRY(validate_attn_dims(B > 0 ? B : 1, S > 0 ? S : 1, h, heads, d, t));
     return TP_OK;
@@ -807,6 +832,7 @@ tp_status tp_layer_forward(const void* X, int B, int S, int h, int heads, int d,
                            const void* bo, const void* ln2_g, const void* ln2_b, const tp_shard* W1,
                            const void* const* b1, const tp_shard* W2, const void* b2, float eps, int causal,
                            void* out, tp_reduce_mode mode, void* ws, size_t ws_bytes, tp_stream_t stream) {
+  ApiRange range("tp_layer_forward");
   const int64_t M = static_cast<int64_t>(B) * S;
   if (mode != TP_REDUCE_FUSED && mode != TP_REDUCE_PARTIALS) return fail(TP_ERR_INVALID_ARG, "unknown mode");
   TP_TRY(validate_attn_dims(B > 0 ? B : 1, S > 0 ? S : 1, h, heads, d, t));
@@ -850,6 +876,7 @@ tp_status tp_layer_forward(const void* X, int B, int S, int h, int heads, int d,
 
 tp_status tp_layernorm_forward(const void* x, tp_dtype in_dtype, const void* gamma, const void* beta, int64_t M,
                                int64_t h, float eps, void* y, tp_dtype out_dtype, tp_stream_t stream) {
+  ApiRange range("tp_layernorm_forward");
   if (in_dtype != TP_BF16 && in_dtype != TP_FP32) return fail(TP_ERR_INVALID_ARG, "unknown input dtype");
   if (out_dtype != TP_BF16 && out_dtype != TP_FP16) return fail(TP_ERR_INVALID_ARG, "unknown output dtype");
   if (M < 0 || h <= 0) return fail(TP_ERR_INVALID_ARG, "bad sizes");
@@ -867,6 +894,7 @@ tp_status tp_layernorm_forward(const void* x, tp_dtype in_dtype, const void* gam
 
 tp_status tp_reduce_partials(const float* P, int t, int64_t M, int64_t h, const void* bias, const void* residual,
                              tp_dtype dtype, void* out, tp_stream_t stream) {
+  ApiRange range("tp_reduce_partials");
   if (dtype != TP_BF16 && dtype != TP_FP32) return fail(TP_ERR_INVALID_ARG, "unknown dtype");
   if (t < 1 || M < 0 || h <= 0) return fail(TP_ERR_INVALID_ARG, "bad sizes");
   if (h % 4) return fail(TP_ERR_UNSUPPORTED, "h %% 4 != 0");
@@ -879,6 +907,7 @@ tp_status tp_reduce_partials(const float* P, int t, int64_t M, int64_t h, const 
 }
 
 tp_status tp_activation_forward(const float* x, float* y, int64_t n, tp_activation act, tp_stream_t stream) {
+  ApiRange range("tp_activation_forward");
   if (n < 0) return fail(TP_ERR_INVALID_ARG, "n must be >= 0");
   if (act != TP_ACT_GELU && act != TP_ACT_RELU) return fail(TP_ERR_INVALID_ARG, "unknown activation %d", act);
   if (n > 0 && (!x || !y)) return fail(TP_ERR_INVALID_ARG, "x or y is NULL");

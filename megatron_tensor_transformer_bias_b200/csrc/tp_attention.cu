@@ -897,7 +897,7 @@ tp_status launch_attention(const AttnArgs& a, cudaStream_t stream) {
     attr_set[dev] |= one ? 1 : 2;
   }
   if (a.S <= 0 || a.B == 0 || a.H - a.head0 <= 0) return TP_OK;
-  trace_before(stream);
+  trace_before(stream, "attention");
   tp_status st;
   if (one) {
     const int nqb = (a.S + BQ - 1) / BQ;

@@ -1094,7 +1094,7 @@ static tp_status launch_gemm_pair(const GemmArgs& a, cudaStream_t stream, const 
   const long long tiles = 1LL * m_tiles * n_tiles * (a.concat ? 1 : a.G);
   if (tiles <= 0) return TP_OK;
   const int nclusters = static_cast<int>(tiles < nclusters_max ? tiles : nclusters_max);
-  trace_before(stream);
+  trace_before(stream, name);
   const tp_status st = launch_ex(gemm_kernel_for(a.epi, opl, true), dim3(2 * nclusters), dim3(THREADS), P_SMEM_BYTES,
                                  stream, 2, a);
   if (st != TP_OK) return st;
@@ -1114,7 +1114,7 @@ tp_status launch_gemm(const GemmArgs& a, cudaStream_t stream, const char* name) 
   const long long tiles = 1LL * m_tiles * n_tiles * (a.concat ? 1 : a.G);
   if (tiles <= 0) return TP_OK;
   const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
-  trace_before(stream);
+  trace_before(stream, name);
   const tp_status st = launch_ex(gemm_kernel_for(a.epi, opl, false), dim3(grid), dim3(THREADS), SMEM_BYTES, stream, 1, a);
   if (st != TP_OK) return st;
   trace_after(stream, name);

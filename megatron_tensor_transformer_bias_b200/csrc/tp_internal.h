@@ -191,7 +191,7 @@ tp_status launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, 
 
 
 // Launch tracing (tp_trace_*): brackets each kernel launch with events.
-void trace_before(cudaStream_t stream);
+void trace_before(cudaStream_t stream, const char* name);
 void trace_after(cudaStream_t stream, const char* name);
 
 }  // namespace tpb

@@ -23,6 +23,8 @@
 #include <atomic>
 #include <cstdio>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "tp_internal.h"
 
 namespace {
@@ -61,11 +63,9 @@ tp_status scratch_address(cudaStream_t stream, void** out) {
   return TP_OK;
 }
 
-}  // namespace
-
-extern "C" tp_status tp_ffn_forward_noalloc(const void* X, int64_t M, int64_t h, int64_t f, int t,
-                                            const tp_shard* W1, const void* const* b1, const tp_shard* W2,
-                                            const void* b2, const void* residual, void* out, tp_stream_t stream) {
+tp_status ffn_noalloc(const void* X, int64_t M, int64_t h, int64_t f, int t, const tp_shard* W1,
+                      const void* const* b1, const tp_shard* W2, const void* b2, const void* residual, void* out,
+                      tp_stream_t stream) {
   if (M < 0 || h <= 0 || f <= 0) return tpb::set_error(TP_ERR_INVALID_ARG, "sizes must be positive (M>=0)");
   if (t < 1 || t > TP_MAX_SHARDS) return tpb::set_error(TP_ERR_INVALID_ARG, "t outside [1, 16]");
   if (!W1 || !W2) return tpb::set_error(TP_ERR_INVALID_ARG, "shard array is NULL");
@@ -89,4 +89,15 @@ extern "C" tp_status tp_ffn_forward_noalloc(const void* X, int64_t M, int64_t h,
   if (c != TP_OK) return c;
   // steps 2-3: out = sum_i act(Z)_i W2_i + b2 + residual, shards summed in one accumulator
   return tp_row_linear_forward(scratch, M, f, h, t, W2, b2, residual, out, TP_REDUCE_FUSED, nullptr, 0, stream);
+}
+
+}  // namespace
+
+extern "C" tp_status tp_ffn_forward_noalloc(const void* X, int64_t M, int64_t h, int64_t f, int t,
+                                            const tp_shard* W1, const void* const* b1, const tp_shard* W2,
+                                            const void* b2, const void* residual, void* out, tp_stream_t stream) {
+  nvtxRangePushA("tp_ffn_forward_noalloc");
+  const tp_status s = ffn_noalloc(X, M, h, f, t, W1, b1, W2, b2, residual, out, stream);
+  nvtxRangePop();
+  return s;
 }

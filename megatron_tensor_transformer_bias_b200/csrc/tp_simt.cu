@@ -288,7 +288,7 @@ tp_status launch_reduce_partials(const float* P, int t, int64_t M, int64_t h, co
   if (blocks > cap) blocks = cap;
   const int g = static_cast<int>(blocks);
   const int key = (out_fp32 ? 4 : 0) | (resid_fp32 ? 2 : 0) | (bias_fp32 ? 1 : 0);
-  trace_before(stream);
+  trace_before(stream, "reduce_partials");
   tp_status st = TP_OK;
   switch (key) {
 #define TP_REDUCE_CASE(K, O, R, B)                                                                              \
@@ -414,7 +414,7 @@ static tp_status launch_layernorm_reg(const void* x, int in_fp32, const void* g,
       : key == 1 ? layernorm_reg_kernel<true, false, NCH>
       : key == 2 ? layernorm_reg_kernel<false, true, NCH>
                  : layernorm_reg_kernel<true, true, NCH>;
-  trace_before(stream);
+  trace_before(stream, "layernorm");
   const tp_status st = launch_ex(kern, dim3(static_cast<unsigned>(M)), dim3(LN_THREADS), 0, stream, 1, x,
                                  static_cast<const uint16_t*>(g), static_cast<const uint16_t*>(b), h, eps,
                                  static_cast<uint16_t*>(y), device_status_ptr());
@@ -445,7 +445,7 @@ tp_status launch_layernorm(const void* x, int in_fp32, const void* g, const void
       return TP_ERR_CUDA;
     attr_set[dev][key] = 1;
   }
-  trace_before(stream);
+  trace_before(stream, "layernorm");
   const tp_status st = launch_ex(kern, dim3(static_cast<unsigned>(M)), dim3(LN_THREADS), smem, stream, 1, x,
                                  static_cast<const uint16_t*>(g), static_cast<const uint16_t*>(b), h, eps,
                                  static_cast<uint16_t*>(y), device_status_ptr());
@@ -470,14 +470,14 @@ tp_status launch_ffn_fp32(const float* X, int64_t M, int64_t h, int64_t f, int t
   // Step 1: Z[:, i*fs:(i+1)*fs] = act(X W1_i + b1_i)
   dim3 blk(SG, SG);
   dim3 g1(static_cast<unsigned>((fs + SG - 1) / SG), static_cast<unsigned>((M + SG - 1) / SG), t);
-  trace_before(stream);
+  trace_before(stream, "f32_col_gemm");
   f32_gemm_kernel<<<g1, blk, 0, stream>>>(X, h, 0, s1, Z, f, fs, 0, static_cast<int>(M), static_cast<int>(fs),
                                           static_cast<int>(h), act);
   if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
   trace_after(stream, "f32_col_gemm");
   // Step 2: P[i] = Z_i W2_i
   dim3 g2(static_cast<unsigned>((h + SG - 1) / SG), static_cast<unsigned>((M + SG - 1) / SG), t);
-  trace_before(stream);
+  trace_before(stream, "f32_row_gemm");
   f32_gemm_kernel<<<g2, blk, 0, stream>>>(Z, f, fs, s2, P, h, 0, M * h, static_cast<int>(M), static_cast<int>(h),
                                           static_cast<int>(fs), ACT_NONE);
   if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
@@ -491,7 +491,7 @@ tp_status launch_act(const float* x, float* y, int64_t n, int act, cudaStream_t 
   int64_t blocks = (n + 255) / 256;
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
   if (blocks > cap) blocks = cap;
-  trace_before(stream);
+  trace_before(stream, "activation");
   act_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(x, y, n, act);
   if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
   trace_after(stream, "activation");
@@ -510,11 +510,11 @@ tp_status launch_colsum(const void* x, int64_t M, int64_t n, int64_t ld, float* 
     const cudaError_t e = cudaMemsetAsync(out, 0, static_cast<size_t>(n) * sizeof(float), stream);
     return e == cudaSuccess ? TP_OK : set_error(TP_ERR_CUDA, cudaGetErrorString(e));
   }
-  trace_before(stream);
+  trace_before(stream, "colsum");
   TP_TRY_LAUNCH(launch_ex(colsum_chunk_kernel, dim3(static_cast<unsigned>((n + CS_COLS - 1) / CS_COLS), chunks),
                           dim3(256), 0, stream, 1, static_cast<const uint16_t*>(x), M, n, ld, part));
   trace_after(stream, "colsum");
-  trace_before(stream);
+  trace_before(stream, "colsum");
   TP_TRY_LAUNCH(launch_ex(colsum_final_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, stream, 1,
                           static_cast<const float*>(part), chunks, n, out));
   trace_after(stream, "colsum");
@@ -522,7 +522,7 @@ tp_status launch_colsum(const void* x, int64_t M, int64_t n, int64_t ld, float* 
 }
 
 tp_status launch_selftest_wait(uint64_t limit_ns, cudaStream_t stream) {
-  trace_before(stream);
+  trace_before(stream, "selftest_wait");
   selftest_wait_kernel<<<1, 32, 0, stream>>>(limit_ns, device_status_ptr());
   if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
   trace_after(stream, "selftest_wait");

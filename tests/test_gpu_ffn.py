@@ -142,6 +142,28 @@ def test_row_linear(mode):
     assert_bf16_close(out, ref, f"row linear {mode}")
 
 
+# Wide fused row layers, every element checked: two blocks of 256 rows x 40 column tiles
+# (more tiles than CTA pairs, a second round of tiles), ragged M, and N = 10176, which is
+# not a multiple of the 256-column tile.
+ROW_WIDE_CASES = [(512, 256, 10240, 2), (300, 128, 10176, 1), (400, 512, 10240, 4)]
+
+
+@pytest.mark.parametrize("M,k,n,t", ROW_WIDE_CASES)
+def test_row_linear_wide_full(M, k, n, t):
+    g = torch.Generator(device=DEV).manual_seed(M + n)
+    A = torch.randn(M, k, generator=g, device=DEV).to(torch.bfloat16)
+    W = (torch.randn(k, n, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    bias = (torch.randn(n, generator=g, device=DEV) * 0.01).to(torch.bfloat16)
+    R = torch.randn(M, n, generator=g, device=DEV).to(torch.bfloat16)
+    out = torch.full((M, n), float("nan"), dtype=torch.bfloat16, device=DEV)
+    tb.tp_row_linear_forward(A, tb.shard_rows(W, t), bias, R, out, mode="fused")
+    assert tb.tp_get_device_status() == tb.TP_OK
+    assert torch.isfinite(out.float()).all(), "an output element was not written"
+    ref = oracle.reduce_partials([to64(A[:, i * k // t:(i + 1) * k // t]) @ to64(W[i * k // t:(i + 1) * k // t])
+                                  for i in range(t)], to64(bias), to64(R))
+    assert_bf16_close(out, ref, f"row linear {M}x{k}x{n} t={t}")
+
+
 ROW_PARTIAL_CASES = [(300, 384, 4), (1, 320, 2), (129, 256, 1), (513, 1024, 8), (2048, 4096, 4)]
 
 
