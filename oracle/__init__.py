@@ -15,7 +15,10 @@ reordering is added beyond what the definitions state.
 The backward pass of the FFN block (gradients of the forward block by the
 chain rule, with the sum over shards of the column layer's input gradient as
 its one reduction) is pinned the same way: a normal-table check of GeLU',
-central finite differences, float64 autograd and sharding invariance.
+central finite differences, float64 autograd and sharding invariance; so is
+the attention sub-layer's backward pass (finite differences of the forward
+oracle, float64 autograd of torch's attention, head-group sharding and
+permutation, closed forms for one-token sequences and a constant V).
 
 Source of the method: the page "Tensor Parallelism > Combining Column and Row
 Parallelism" (mbrenndoerfer.com), cited below as [TP-CR] with its numbered
@@ -43,4 +46,7 @@ from .tp_block import (  # noqa: F401
     relu_grad,
     ffn_backward,
     ffn_backward_sharded,
+    attention_heads_backward,
+    attn_backward,
+    attn_backward_sharded,
 )

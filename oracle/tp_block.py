@@ -326,3 +326,112 @@ def ffn_backward_sharded(X, shards: Iterable[Tuple], dY, act="gelu"):
         part = dZ_i @ W1_i.T
         dX = part if dX is None else dX + part
     return dX, dW1, db1, dW2, dY.sum(axis=0)
+
+
+# --------------------------------------------------------------------------
+# Backward pass of the attention sub-layer.  Same reading as the FFN block's:
+# the chain rule back through the output projection (row-parallel: its input
+# gradient dO_i = dY Wo_i^T is local to head group i), per-head attention
+# (heads are independent) and the QKV projection (column-parallel: the input
+# gradient dX = sum_i dQKV_i Wqkv_i^T is the one reduction over groups).
+# --------------------------------------------------------------------------
+def attention_heads_backward(Q, K, V, dO, causal):
+    """Gradients of O = softmax(Q K^T / sqrt(d), masked) V for one sequence, head by head.
+
+    Q, K, V, dO [S, Hn, d].  For each head, with s = Q K^T / sqrt(d) (masked
+    scores -inf) and P = softmax over keys:
+        dV = P^T dO,   dP = dO V^T,
+        dS = P * (dP - rowsum(P * dP))      (the softmax Jacobian applied row by row),
+        dQ = dS K / sqrt(d),   dK = dS^T Q / sqrt(d).
+    Returns dQ, dK, dV [S, Hn, d].
+    """
+    Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
+    S, Hn, d = Q.shape
+    scale = 1.0 / math.sqrt(d)
+    keep = (np.arange(S)[None, :] <= np.arange(S)[:, None]) if causal else np.ones((S, S), bool)
+    dQ, dK, dV = (np.empty_like(Q) for _ in range(3))
+    for g in range(Hn):
+        s = np.where(keep, (Q[:, g, :] @ K[:, g, :].T) * scale, -np.inf)
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        p = p / p.sum(axis=1, keepdims=True)
+        dV[:, g, :] = p.T @ dO[:, g, :]
+        dp = dO[:, g, :] @ V[:, g, :].T
+        ds = p * (dp - np.sum(p * dp, axis=1, keepdims=True))
+        dQ[:, g, :] = ds @ K[:, g, :] * scale
+        dK[:, g, :] = ds.T @ Q[:, g, :] * scale
+    return dQ, dK, dV
+
+
+def attn_backward(X, Wq, Wk, Wv, Wo, dY, B, S, H, d, causal=True, bqkv=None):
+    """Gradients of out = concat_h(attention_h) Wo + bo + R given dY = dL/d(out).
+
+    Returns a dict with dX (through the attention path only; with R = X the
+    caller's total input gradient is dX + dY), dWq, dWk, dWv, dbq, dbk, dbv,
+    dWo and dbo:
+        Q = X Wq (+ bq), K = X Wk (+ bk), V = X Wv (+ bv),  O = attention(Q, K, V)
+        dWo = O^T dY,   dbo = sum over rows of dY,   dO = dY Wo^T
+        dQ, dK, dV = attention_heads_backward(Q, K, V, dO) per sequence
+        dWq = X^T dQ (likewise K, V),  dbq = sum over rows of dQ (likewise K, V)
+        dX = dQ Wq^T + dK Wk^T + dV Wv^T
+    """
+    X, Wq, Wk, Wv, Wo, dY = _f64(X), _f64(Wq), _f64(Wk), _f64(Wv), _f64(Wo), _f64(dY)
+    M = B * S
+    Q, K, V = X @ Wq, X @ Wk, X @ Wv
+    if bqkv is not None:
+        Q, K, V = Q + _f64(bqkv[0]), K + _f64(bqkv[1]), V + _f64(bqkv[2])
+    O = np.empty((M, H * d), dtype=F64)
+    for b in range(B):
+        sl = slice(b * S, (b + 1) * S)
+        O[sl] = attention_heads(Q[sl].reshape(S, H, d), K[sl].reshape(S, H, d), V[sl].reshape(S, H, d),
+                                causal).reshape(S, H * d)
+    dO = dY @ Wo.T
+    dQ, dK, dV = (np.empty((M, H * d), dtype=F64) for _ in range(3))
+    for b in range(B):
+        sl = slice(b * S, (b + 1) * S)
+        gq, gk, gv = attention_heads_backward(Q[sl].reshape(S, H, d), K[sl].reshape(S, H, d),
+                                              V[sl].reshape(S, H, d), dO[sl].reshape(S, H, d), causal)
+        dQ[sl], dK[sl], dV[sl] = gq.reshape(S, H * d), gk.reshape(S, H * d), gv.reshape(S, H * d)
+    return {"dX": dQ @ Wq.T + dK @ Wk.T + dV @ Wv.T,
+            "dWq": X.T @ dQ, "dWk": X.T @ dK, "dWv": X.T @ dV,
+            "dbq": dQ.sum(axis=0), "dbk": dK.sum(axis=0), "dbv": dV.sum(axis=0),
+            "dWo": O.T @ dY, "dbo": dY.sum(axis=0)}
+
+
+def attn_backward_sharded(X, Wqkv_shards, Wo_shards, dY, B, S, Hg, d, causal=True, bqkv_shards=None):
+    """The backward pass head group by head group, for shards i = 0..t-1 holding
+    Wqkv_i [h, 3*Hg*d] = [Q heads | K heads | V heads] (optional bias bqkv_i) and Wo_i [Hg*d, h]:
+
+    * recompute QKV_i = X Wqkv_i (+ bqkv_i) and the group's attention output O_i (local);
+    * dWo_i = O_i^T dY and dO_i = dY Wo_i^T (the row-parallel projection's gradients, local);
+    * dQKV_i = [dQ | dK | dV] of the group's heads (local; heads are independent);
+    * dWqkv_i = X^T dQKV_i, dbqkv_i = column sums of dQKV_i (local);
+    * dX = sum_i dQKV_i Wqkv_i^T, in the order 0..t-1 (the reduction);
+    * dbo = column sums of dY, once.
+
+    Returns (dX, [dWqkv_i], [dbqkv_i], [dWo_i], dbo)."""
+    X, dY = _f64(X), _f64(dY)
+    M, n = B * S, Hg * d
+    dX = None
+    dWqkv, dbqkv, dWo = [], [], []
+    for i, (Wqkv_i, Wo_i) in enumerate(zip(Wqkv_shards, Wo_shards)):
+        Wqkv_i, Wo_i = _f64(Wqkv_i), _f64(Wo_i)
+        QKV = X @ Wqkv_i
+        if bqkv_shards is not None and bqkv_shards[i] is not None:
+            QKV = QKV + _f64(bqkv_shards[i])
+        O_i = np.empty((M, n), dtype=F64)
+        dQKV = np.empty((M, 3 * n), dtype=F64)
+        dO_i = dY @ Wo_i.T
+        for b in range(B):
+            sl = slice(b * S, (b + 1) * S)
+            q = QKV[sl, 0:n].reshape(S, Hg, d)
+            k = QKV[sl, n:2 * n].reshape(S, Hg, d)
+            v = QKV[sl, 2 * n:3 * n].reshape(S, Hg, d)
+            O_i[sl] = attention_heads(q, k, v, causal).reshape(S, n)
+            gq, gk, gv = attention_heads_backward(q, k, v, dO_i[sl].reshape(S, Hg, d), causal)
+            dQKV[sl] = np.concatenate([gq.reshape(S, n), gk.reshape(S, n), gv.reshape(S, n)], axis=1)
+        dWo.append(O_i.T @ dY)
+        dWqkv.append(X.T @ dQKV)
+        dbqkv.append(dQKV.sum(axis=0))
+        part = dQKV @ Wqkv_i.T
+        dX = part if dX is None else dX + part
+    return dX, dWqkv, dbqkv, dWo, dY.sum(axis=0)

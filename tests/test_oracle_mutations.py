@@ -132,3 +132,48 @@ def test_input_gradient_missing_a_shard_is_caught(monkeypatch):
         return dX - dX_l if len(shards) > 1 else dX, dW1, db1, dW2, db2
     monkeypatch.setattr(oracle, "ffn_backward_sharded", drop_last_shard_from_dx)
     _expect_fail(pins.check_ffn_backward_sharding)
+
+
+def test_attention_backward_without_row_correction_is_caught(monkeypatch):
+    # dS = P * dP, the softmax Jacobian's rowsum(P * dP) term dropped
+    def bad(Q, K, V, dO, causal):
+        Q, K, V, dO = (np.asarray(x, float) for x in (Q, K, V, dO))
+        S, Hn, d = Q.shape
+        scale = 1.0 / math.sqrt(d)
+        keep = (np.arange(S)[None, :] <= np.arange(S)[:, None]) if causal else np.ones((S, S), bool)
+        dQ, dK, dV = (np.empty_like(Q) for _ in range(3))
+        for g in range(Hn):
+            s = np.where(keep, (Q[:, g] @ K[:, g].T) * scale, -np.inf)
+            p = np.exp(s - s.max(axis=1, keepdims=True))
+            p = p / p.sum(axis=1, keepdims=True)
+            dV[:, g] = p.T @ dO[:, g]
+            ds = p * (dO[:, g] @ V[:, g].T)
+            dQ[:, g] = ds @ K[:, g] * scale
+            dK[:, g] = ds.T @ Q[:, g] * scale
+        return dQ, dK, dV
+    monkeypatch.setattr(tb, "attention_heads_backward", bad)
+    monkeypatch.setattr(oracle, "attention_heads_backward", bad)
+    _expect_fail(lambda: pins.check_attn_backward_finite_differences(True))
+
+
+def test_attention_backward_transposed_dk_is_caught(monkeypatch):
+    real = tb.attention_heads_backward
+
+    def swapped(Q, K, V, dO, causal):
+        dQ, dK, dV = real(Q, K, V, dO, causal)
+        return dK, dQ, dV
+    monkeypatch.setattr(tb, "attention_heads_backward", swapped)
+    _expect_fail(lambda: pins.check_attn_backward_finite_differences(True))
+
+
+def test_attention_backward_group_sum_missing_a_shard_is_caught(monkeypatch):
+    real = tb.attn_backward_sharded
+
+    def first_shard_only_dx(X, Wqkv, Wo, dY, B, S, Hg, d, causal=True, bqkv_shards=None):
+        out = list(real(X, Wqkv, Wo, dY, B, S, Hg, d, causal, bqkv_shards))
+        if len(Wqkv) > 1:
+            out[0] = real(X, Wqkv[:1], Wo[:1], dY, B, S, Hg, d, causal,
+                          None if bqkv_shards is None else bqkv_shards[:1])[0]
+        return tuple(out)
+    monkeypatch.setattr(oracle, "attn_backward_sharded", first_shard_only_dx)
+    _expect_fail(pins.check_attn_backward_sharding)

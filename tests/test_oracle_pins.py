@@ -503,3 +503,128 @@ def test_ffn_backward_special_cases():
     A = oracle.gelu(X @ W1 + b1)
     np.testing.assert_allclose(g["dW2"], A.T @ dY, rtol=1e-14)
     np.testing.assert_allclose(g["db2"], dY.sum(0), rtol=1e-14)
+
+
+# ------------------------------------------------------------------ attention backward
+def _tiny_attn_backward_case(seed=31, B=2, S=5, h=8, H=2, d=4):
+    rng = np.random.default_rng(seed)
+    return {"X": rng.standard_normal((B * S, h)), "Wq": rng.standard_normal((h, H * d)) * 0.5,
+            "Wk": rng.standard_normal((h, H * d)) * 0.5, "Wv": rng.standard_normal((h, H * d)) * 0.5,
+            "Wo": rng.standard_normal((H * d, h)) * 0.5, "bo": rng.standard_normal(h) * 0.3,
+            "bq": rng.standard_normal(H * d) * 0.3, "bk": rng.standard_normal(H * d) * 0.3,
+            "bv": rng.standard_normal(H * d) * 0.3, "dY": rng.standard_normal((B * S, h))}
+
+
+def check_attn_backward_finite_differences(causal=True):
+    """Every gradient entry of L = sum(dY * out) against a central difference of the
+    forward oracle (attn_forward), which shares no code with the backward."""
+    B, S, h, H, d = 2, 5, 8, 2, 4
+    a = _tiny_attn_backward_case(B=B, S=S, h=h, H=H, d=d)
+    g = oracle.attn_backward(a["X"], a["Wq"], a["Wk"], a["Wv"], a["Wo"], a["dY"], B, S, H, d, causal,
+                             bqkv=(a["bq"], a["bk"], a["bv"]))
+    names = ["X", "Wq", "Wk", "Wv", "Wo", "bo", "bq", "bk", "bv"]
+
+    def loss(p):
+        out = oracle.attn_forward(p["X"], p["Wq"], p["Wk"], p["Wv"], p["Wo"], p["bo"], None, B, S, H, d,
+                                  causal, bqkv=(p["bq"], p["bk"], p["bv"]))
+        return float(np.sum(a["dY"] * out))
+
+    eps = 1e-6
+    for name in names:
+        fd = np.zeros_like(a[name])
+        for idx in np.ndindex(a[name].shape):
+            up = dict(a); dn = dict(a)
+            up[name] = a[name].copy(); dn[name] = a[name].copy()
+            up[name][idx] += eps
+            dn[name][idx] -= eps
+            fd[idx] = (loss(up) - loss(dn)) / (2 * eps)
+        np.testing.assert_allclose(g["d" + name], fd, rtol=1e-6, atol=1e-7, err_msg=name)
+
+
+def test_attn_backward_finite_differences():
+    check_attn_backward_finite_differences(True)
+    check_attn_backward_finite_differences(False)
+
+
+def test_attn_backward_matches_float64_autograd():
+    """Against autograd through torch's own scaled_dot_product_attention in float64."""
+    B, S, h, H, d = 2, 7, 16, 4, 4
+    a = _tiny_attn_backward_case(seed=32, B=B, S=S, h=h, H=H, d=d)
+    for causal in (True, False):
+        t = {k: torch.tensor(a[k], dtype=torch.float64, requires_grad=True)
+             for k in ("X", "Wq", "Wk", "Wv", "Wo", "bo", "bq", "bk", "bv")}
+        X = t["X"].view(B, S, h)
+        q = (X @ t["Wq"] + t["bq"]).view(B, S, H, d).transpose(1, 2)
+        k = (X @ t["Wk"] + t["bk"]).view(B, S, H, d).transpose(1, 2)
+        v = (X @ t["Wv"] + t["bv"]).view(B, S, H, d).transpose(1, 2)
+        o = F.scaled_dot_product_attention(q, k, v, is_causal=causal).transpose(1, 2).reshape(B * S, H * d)
+        out = o @ t["Wo"] + t["bo"]
+        out.backward(torch.tensor(a["dY"]))
+        g = oracle.attn_backward(a["X"], a["Wq"], a["Wk"], a["Wv"], a["Wo"], a["dY"], B, S, H, d, causal,
+                                 bqkv=(a["bq"], a["bk"], a["bv"]))
+        for name in t:
+            np.testing.assert_allclose(g["d" + name], t[name].grad.numpy(), rtol=1e-11, atol=1e-12,
+                                       err_msg=f"{name} causal={causal}")
+
+
+def check_attn_backward_sharding():
+    """Head group by head group (local projection gradients, one ordered sum for dX) equals
+    the unsharded chain rule for every t dividing H, and permuting the groups across shards
+    (with their Wo rows) permutes the per-shard gradients and leaves dX, dbo unchanged."""
+    B, S, h, H, d = 2, 6, 16, 4, 4
+    a = _tiny_attn_backward_case(seed=33, B=B, S=S, h=h, H=H, d=d)
+    g = oracle.attn_backward(a["X"], a["Wq"], a["Wk"], a["Wv"], a["Wo"], a["dY"], B, S, H, d, True,
+                             bqkv=(a["bq"], a["bk"], a["bv"]))
+    for t, perm in ((1, None), (2, None), (4, None), (4, [2, 0, 3, 1])):
+        n = (H // t) * d
+        order = list(range(t)) if perm is None else perm
+        Wqkv, Wo, bqkv = [], [], []
+        for i in order:
+            cols = slice(i * n, (i + 1) * n)
+            Wqkv.append(np.concatenate([a["Wq"][:, cols], a["Wk"][:, cols], a["Wv"][:, cols]], axis=1))
+            bqkv.append(np.concatenate([a["bq"][cols], a["bk"][cols], a["bv"][cols]]))
+            Wo.append(a["Wo"][cols, :])
+        dX, dWqkv, dbqkv, dWo, dbo = oracle.attn_backward_sharded(a["X"], Wqkv, Wo, a["dY"], B, S, H // t, d,
+                                                                  True, bqkv_shards=bqkv)
+        np.testing.assert_allclose(dX, g["dX"], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(dbo, g["dbo"], rtol=0, atol=1e-12)
+        for j, i in enumerate(order):
+            cols = slice(i * n, (i + 1) * n)
+            want = np.concatenate([g["dWq"][:, cols], g["dWk"][:, cols], g["dWv"][:, cols]], axis=1)
+            np.testing.assert_allclose(dWqkv[j], want, rtol=0, atol=1e-12)
+            want_b = np.concatenate([g["dbq"][cols], g["dbk"][cols], g["dbv"][cols]])
+            np.testing.assert_allclose(dbqkv[j], want_b, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(dWo[j], g["dWo"][cols, :], rtol=0, atol=1e-12)
+
+
+def test_attn_backward_sharding():
+    check_attn_backward_sharding()
+
+
+def test_attn_backward_special_cases():
+    a = _tiny_attn_backward_case(seed=34)
+    rng = np.random.default_rng(35)
+    # one-token sequences: softmax over a single key is 1, so no gradient reaches Q or K,
+    # and dV = dO
+    S, Hn, d = 1, 3, 4
+    Q, K, V, dO = (rng.standard_normal((S, Hn, d)) for _ in range(4))
+    dQ, dK, dV = oracle.attention_heads_backward(Q, K, V, dO, True)
+    assert not np.any(dQ) and not np.any(dK)
+    np.testing.assert_allclose(dV, dO, rtol=0, atol=0)
+    # V constant across keys: O does not depend on the scores, so dQ = dK = 0 and dV is the
+    # column sums of P weighted by dO (each row of P sums to 1: sum over keys of dV = sum of dO)
+    S = 6
+    Q, K, dO = (rng.standard_normal((S, Hn, d)) for _ in range(3))
+    V = np.broadcast_to(rng.standard_normal((1, Hn, d)), (S, Hn, d)).copy()
+    for causal in (True, False):
+        dQ, dK, dV = oracle.attention_heads_backward(Q, K, V, dO, causal)
+        np.testing.assert_allclose(dQ, 0, atol=1e-14)
+        np.testing.assert_allclose(dK, 0, atol=1e-14)
+        np.testing.assert_allclose(dV.sum(axis=0), dO.sum(axis=0), rtol=1e-13, atol=1e-13)
+    # causal: the last key is seen by the last query only, so its dK / dV come from that row
+    dQ, dK, dV = oracle.attention_heads_backward(Q, K, rng.standard_normal((S, Hn, d)), dO, True)
+    assert np.all(np.isfinite(dK))
+    # dY = 0: every gradient is zero
+    z = oracle.attn_backward(a["X"], a["Wq"], a["Wk"], a["Wv"], a["Wo"], np.zeros_like(a["dY"]), 2, 5, 2, 4)
+    for v in z.values():
+        assert not np.any(v)
