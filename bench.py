@@ -446,6 +446,92 @@ class Attn(Workload):
         return len(rows), self.flops * len(rows) / w.M
 
 
+class AttnBwd(Workload):
+    """One backward pass of the attention sub-layer (tp_attn_backward).  FLOPs: the model
+    count, 16*M*h*H*d for the two projections' weight and input gradients plus
+    8*B*H*d*pairs for dV, dP, dQ and dK (pairs = S(S+1)/2 causal); the call also
+    recomputes Q, K, V, O and the scores (reported as executed_flops_per_step).  The
+    per-step input is X and dY, stacked."""
+    ref_rows = 8
+
+    def __init__(self, w):
+        self.w = w
+        self.name = "attn_bwd_" + w.name[len("attn_"):]
+        M, h, H, d, B, S = w.M, w.h, w.H, w.d, w.B, w.S
+        self.pairs = S * (S + 1) // 2 if w.causal else S * S
+        self.flops = 16 * M * h * H * d + 8 * B * H * d * self.pairs
+        blocks = (S + 127) // 128
+        # the backward kernels work in whole 128 x 128 blocks (diagonal ones included)
+        bpairs = (blocks * (blocks + 1) // 2 if w.causal else blocks * blocks) * 128 * 128
+        self.kernel_amount = {
+            "gemm_qkv": ("tensor", 2 * M * h * 3 * H * d, "FLOP"),
+            "attention": ("tensor", 4 * B * H * d * self.pairs, "FLOP"),
+            "gemm_attn_bwd_dwo": ("tensor", 2 * M * H * d * h, "FLOP"),
+            "gemm_attn_bwd_do": ("tensor", 2 * M * h * H * d, "FLOP"),
+            "attn_bwd_rowdot": ("hbm", M * H * d * 4, "B"),
+            "attn_bwd_dkdv": ("tensor", 8 * B * H * d * bpairs, "FLOP"),
+            "attn_bwd_dq": ("tensor", 6 * B * H * d * bpairs, "FLOP"),
+            "gemm_attn_bwd_dwqkv": ("tensor", 2 * M * h * 3 * H * d, "FLOP"),
+            "gemm_attn_bwd_dx": ("tensor", 2 * M * 3 * H * d * h, "FLOP"),
+        }
+        self.executed = 22 * M * h * H * d + (4 * self.pairs + 14 * bpairs) * B * H * d
+
+    def setup(self, dev, rank):
+        import torch
+        from megatron_tensor_transformer_bias_b200 import inputs
+        from megatron_tensor_transformer_bias_b200 import tpblock as tb
+        w = self.w
+        a = inputs.attn_inputs(w.B, w.S, w.h, w.H, w.d, seed=rank, device=dev)
+        g = torch.Generator(device=dev).manual_seed(9100 + 7919 * rank)
+        a["dY"] = torch.randn(w.M, w.h, generator=g, device=dev).to(torch.bfloat16)
+        self.p = a
+        self.packed = inputs.pack_qkv(a["Wq"], a["Wk"], a["Wv"], w.t, w.H, w.d)
+        self.Wqkv = tb.shard_columns(self.packed, w.t)
+        self.Wo = tb.shard_rows(a["Wo"], w.t)
+        Hd = w.H * w.d
+        self.dWqkv = torch.empty(w.h, 3 * Hd, dtype=torch.float32, device=dev)
+        self.dWo = torch.empty(Hd, w.h, dtype=torch.float32, device=dev)
+        self.dbqkv = torch.empty(3 * Hd, dtype=torch.float32, device=dev)
+        self.dbo = torch.empty(w.h, dtype=torch.float32, device=dev)
+        self.ws = tb.workspace(tb.tp_attn_backward_workspace_bytes(w.B, w.S, w.h, w.H, w.d, w.t), dev)
+        self.tb = tb
+        return torch.stack([a["X"], a["dY"]])
+
+    def make_out(self, X):
+        import torch
+        return torch.empty_like(X[0])
+
+    def step(self, XdY, dX, stream):
+        w = self.w
+        self.tb.tp_attn_backward(XdY[0], w.B, w.S, w.H, w.d, self.Wqkv, None, self.Wo, XdY[1], dX, self.dWqkv,
+                                 self.dWo, self.dbqkv, self.dbo, dX_add=XdY[1], causal=w.causal, ws=self.ws,
+                                 stream=stream)
+
+    def config(self):
+        w = self.w
+        return {"workload": self.name, "B": w.B, "S": w.S, "h": w.h, "heads": w.H, "d": w.d, "t": w.t,
+                "causal": w.causal, "dtype": "bf16",
+                "gradients": "dX bf16 (+ dY, the residual path); dWqkv, dWo, dbqkv, dbo fp32 kept on the device",
+                "executed_flops_per_step": self.executed, "e2e_io": "X and dY in, dX out"}
+
+    def oracle_setup(self, src):
+        return {k: _to64(v) for k, v in src.items()}
+
+    def oracle_rows(self, st, rng, n):
+        """The oracle's backward of one random head over one random sequence (its projection
+        columns and rows and its attention), credited 1/(B*H) of the workload's FLOPs."""
+        import numpy as np
+        import oracle
+        w = self.w
+        b, head = int(rng.integers(w.B)), int(rng.integers(w.H))
+        d = w.d
+        cols = slice(head * d, (head + 1) * d)
+        Wqkv_h = np.concatenate([st["Wq"][:, cols], st["Wk"][:, cols], st["Wv"][:, cols]], axis=1)
+        sl = slice(b * w.S, (b + 1) * w.S)
+        oracle.attn_backward_sharded(st["X"][sl], [Wqkv_h], [st["Wo"][cols]], st["dY"][sl], 1, w.S, 1, d, w.causal)
+        return 1, self.flops / (w.B * w.H)
+
+
 class Layer(Workload):
     ref_rows = 8
 
@@ -525,7 +611,8 @@ def make_workloads(args):
                Layer(configs.LAYER_S2048_H8192, "fused")]
         if args.impl != "reference":   # the oracle's sweep sample needs tens of GB of fp64 weights per step
             out += [sweep(22528, 1), sweep(22528, 8)]
-        out += [FFNBwd(configs.HEADLINE), ffn(4, "partials"), ffn(4, "fused", headline=True)]
+        out += [FFNBwd(configs.HEADLINE), AttnBwd(configs.ATTN_B2_S2048), ffn(4, "partials"),
+                ffn(4, "fused", headline=True)]
         return out
     if wl == "bwd":
         return [FFNBwd(configs.ffn_2048x4096x16384(args.t) if args.t != 4 else configs.HEADLINE)]
@@ -539,6 +626,8 @@ def make_workloads(args):
         return [sweep(h, t) for h in hs for t in ts]
     if wl == "attn":
         return [Attn(configs.ATTN_B2_S2048, args.mode)]
+    if wl == "attn_bwd":
+        return [AttnBwd(configs.ATTN_B2_S2048)]
     if wl == "layer":
         return [Layer(configs.LAYER_S2048_H8192, args.mode)]
     raise ValueError(wl)
@@ -562,10 +651,15 @@ def cpu_baseline(wl, st, target_s=10.0, rows_per_call=64):
         dt = time.perf_counter() - t0
         if dt >= target_s:
             break
-    out = {"value": round(flops / dt / 1e12, 5), "unit": "TFLOP/s", "kind": "oracle",
-           "sample": f"{calls} oracle call(s) of {min(rows_per_call, wl.w.M)} token rows each ({rows} rows of "
-                     f"{wl.w.M}) of {wl.name}, fp64 numpy/OpenBLAS, {dt:.1f} s wall; credited rows/M of the "
-                     f"workload's FLOPs"}
+    if isinstance(wl, AttnBwd):
+        sample = (f"{calls} oracle call(s) of one head over one sequence each ({calls} of the {wl.w.B * wl.w.H} "
+                  f"head-sequences) of {wl.name}, fp64 numpy/OpenBLAS, {dt:.1f} s wall; credited 1/(B*H) of the "
+                  f"workload's FLOPs per call")
+    else:
+        sample = (f"{calls} oracle call(s) of {min(rows_per_call, wl.w.M)} token rows each ({rows} rows of "
+                  f"{wl.w.M}) of {wl.name}, fp64 numpy/OpenBLAS, {dt:.1f} s wall; credited rows/M of the "
+                  f"workload's FLOPs")
+    out = {"value": round(flops / dt / 1e12, 5), "unit": "TFLOP/s", "kind": "oracle", "sample": sample}
     out.update(_host())
     return out
 
@@ -582,6 +676,10 @@ def run_reference(args, wls):
             import torch
             src = inputs.ffn_inputs(w.M, w.h, w.f, "bf16", seed=0, device="cpu")
             src["dY"] = torch.randn(w.M, w.h, generator=torch.Generator().manual_seed(9000)).to(torch.bfloat16)
+        elif isinstance(wl, AttnBwd):
+            import torch
+            src = inputs.attn_inputs(w.B, w.S, w.h, w.H, w.d, seed=0, device="cpu")
+            src["dY"] = torch.randn(w.M, w.h, generator=torch.Generator().manual_seed(9100)).to(torch.bfloat16)
         elif isinstance(wl, FFN):
             src = inputs.ffn_inputs(w.M, w.h, w.f, w.dtype, seed=0, device="cpu")
         elif isinstance(wl, Attn):
@@ -602,6 +700,9 @@ def run_reference(args, wls):
         value = flops / dt / 1e12
         sample = (f"{n} of {w.M} token rows of {wl.name} per step, fp64 numpy/OpenBLAS; credited rows/M of the "
                   f"workload's FLOPs")
+        if isinstance(wl, AttnBwd):
+            sample = (f"one head over one sequence of {wl.name} per step, fp64 numpy/OpenBLAS; credited 1/(B*H) of "
+                      f"the workload's FLOPs")
         cb = {"value": value, "unit": "TFLOP/s", "kind": "oracle", "sample": sample}
         cb.update(_host())
         line = {"metric": wl.metric(), "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
@@ -793,7 +894,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["all", "ffn", "bwd", "attn", "layer", "sweep", "fp32"], default="all")
+    ap.add_argument("--workload", choices=["all", "ffn", "bwd", "attn", "attn_bwd", "layer", "sweep", "fp32"],
+                    default="all")
     ap.add_argument("--t", type=int, default=4)
     ap.add_argument("--h", default="22528", help="sweep hidden size, or 'all'")
     ap.add_argument("--mode", choices=["fused", "partials"], default="fused")

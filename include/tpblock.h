@@ -252,6 +252,49 @@ TP_API tp_status tp_attn_forward(const void* X, int B, int S, int h, int heads, 
                           int causal, void* out, tp_reduce_mode mode, void* ws, size_t ws_bytes,
                           tp_stream_t stream);
 
+/* ------------------------------------------------------------------ attention sub-layer, backward pass
+ * Gradients of tp_attn_forward's output for the upstream gradient dY, by the
+ * chain rule read with [TP-CR]'s column/row pairing (paragraphs on multi-head
+ * attention and head independence): the output projection is row-parallel, so
+ * its input gradient dO_i = dY Wo_i^T is local to head group i; each head's
+ * attention gradients depend on that head only; the QKV projection is
+ * column-parallel, so its input gradient dX = sum_i dQKV_i Wqkv_i^T is the
+ * backward pass's one sum over groups (taken in one accumulator).
+ *
+ *   Q, K, V = X Wqkv_i (+ bqkv_i), O = attention(Q, K, V)   (recomputed from X,
+ *                                      with each softmax row's log-sum-exp)
+ *   dWo_i = O_i^T dY,   dbo = column sums of dY,   dO_i = dY Wo_i^T
+ *   per head: P = softmax rows, dV = P^T dO, dP = dO V^T,
+ *             dS = P * (dP - rowsum(dO * O)), dQ = dS K / sqrt(d), dK = dS^T Q / sqrt(d)
+ *   dWqkv_i = X^T dQKV_i,   dbqkv_i = column sums of dQKV_i   (dQKV_i = [dQ | dK | dV] of group i)
+ *   dX = sum_i dQKV_i Wqkv_i^T (+ dX_add)
+ *
+ *  X, Wqkv, bqkv, Wo, causal  as in tp_attn_forward, bf16 only (TP_BF16 shards).
+ *  dY       [B*S, h] bf16, contiguous.
+ *  dX_add   [B*S, h] bf16 or NULL, added to dX (pass dY when the forward's
+ *           residual was X).
+ *  dX       [B*S, h] bf16 out; must not alias X, dY or dX_add.
+ *  dWqkv    [h, 3*heads*d] fp32 out, contiguous: group i's gradient is the column
+ *           block [i*3*Hg*d, (i+1)*3*Hg*d) in Wqkv[i]'s [Q | K | V] order.
+ *  dbqkv    [3*heads*d] fp32 out or NULL, same column order.
+ *  dWo      [heads*d, h] fp32 out, contiguous: group i's rows [i*Hg*d, (i+1)*Hg*d).
+ *  dbo      [h] fp32 out or NULL.
+ *  ws       tp_attn_backward_workspace_bytes(...) bytes, 256-byte aligned: Q, K, V,
+ *           O (fp16 / bf16), dO (fp16), dQKV (bf16), the rows' log-sum-exp and
+ *           rowsum(dO * O) (fp32) and the column sums' scratch.
+ * The attention gradients' tensor-core operands (P, dS, dO, Q, K, V) are fp16
+ * with fp32 accumulation; a P or dS value above 65504 sets TP_ERR_RANGE.  The
+ * sums over rows, key blocks, query blocks and groups run in a fixed order:
+ * results are bitwise reproducible on devices with the same SM count.  B*S == 0
+ * zeroes dWqkv, dbqkv, dWo, dbo.  Limits: d == 128, heads % t == 0.
+ */
+TP_API size_t tp_attn_backward_workspace_bytes(int B, int S, int h, int heads, int d, int t);
+TP_API tp_status tp_attn_backward(const void* X, int B, int S, int h, int heads, int d, int t,
+                                  const tp_shard* Wqkv, const void* const* bqkv, const tp_shard* Wo,
+                                  const void* dY, const void* dX_add, int causal, void* dX, float* dWqkv,
+                                  float* dbqkv, float* dWo, float* dbo, void* ws, size_t ws_bytes,
+                                  tp_stream_t stream);
+
 /* ------------------------------------------------------------------ pre-LN layer
  * [TP-CR], the paragraph on two reductions per layer, in pre-LN order:
  *   h1  = X + Attn(LN1(X))            (h1 kept in fp32 inside the workspace)

@@ -237,6 +237,24 @@ tp_status make_tmap_attn(CUtensorMap* map, const void* base, int BH, int S, int 
                            static_cast<uint64_t>(S) * d * 2, 64, box_rows);
 }
 
+// [B*S, H*d] fp16 (token rows, head-major columns) seen as (d, H, S, B): box {64, 1, 128, 1}
+// is 128 rows of one head's 64 columns, the same shared-memory tile as make_tmap_attn's.
+tp_status make_tmap_rows_by_head(CUtensorMap* map, const void* base, int B, int S, int H, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(S),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2,
+                           static_cast<cuuint64_t>(S) * H * d * 2};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled(4d) failed (%d)", static_cast<int>(r));
+  return TP_OK;
+}
+
 }  // namespace tpb
 
 using namespace tpb;
@@ -639,6 +657,164 @@ tp_status attn_bf16(const void* X, int B, int S, int h, int H, int d, int t, con
                  stream);
 }
 
+// ---------------------------------------------------------------- attention backward
+struct AttnBwdWs {
+  AttnWs fwd;          // q, k, v, o as in the forward
+  uint16_t* dO;        // [M, H*d] fp16
+  uint16_t* dqkv;      // [M, 3*H*d] bf16, head groups' [dQ | dK | dV] column blocks
+  float* lse;          // [B*H][S_pad]
+  float* Dv;           // [B*H][S_pad]
+  float* colsum;       // column-sum scratch
+};
+
+int64_t attn_s_pad(int64_t S) { return (S + 127) / 128 * 128; }
+
+size_t attn_bwd_ws_bytes(int64_t B, int64_t S, int64_t h, int64_t H, int64_t d) {
+  const size_t qkv = align_up(static_cast<size_t>(B) * S * H * d * 2);
+  const size_t vec = align_up(static_cast<size_t>(B) * H * attn_s_pad(S) * 4);
+  const int64_t cs = 3 * H * d > h ? 3 * H * d : h;
+  return 4 * qkv + qkv + 3 * qkv + 2 * vec + align_up(colsum_workspace_bytes(B * S, cs));
+}
+
+AttnBwdWs attn_bwd_ws_layout(void* ws, int64_t B, int64_t S, int64_t H, int64_t d) {
+  const size_t qkv = align_up(static_cast<size_t>(B) * S * H * d * 2);
+  const size_t vec = align_up(static_cast<size_t>(B) * H * attn_s_pad(S) * 4);
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  AttnBwdWs w;
+  w.fwd = attn_ws_layout(ws, B, S, H, d);
+  w.dO = reinterpret_cast<uint16_t*>(p + 4 * qkv);
+  w.dqkv = reinterpret_cast<uint16_t*>(p + 5 * qkv);
+  w.lse = reinterpret_cast<float*>(p + 8 * qkv);
+  w.Dv = reinterpret_cast<float*>(p + 8 * qkv + vec);
+  w.colsum = reinterpret_cast<float*>(p + 8 * qkv + 2 * vec);
+  return w;
+}
+
+// Gradients of the attention sub-layer by the chain rule, shard (head group) by shard:
+// recompute Q, K, V and O (with the softmax rows' log2-sum-exp), then the row-parallel
+// projection's gradients (local per group), the attention gradients (per head), the
+// column-parallel projection's weight gradients (local) and its input gradient (the sum
+// over groups, in one accumulator).
+tp_status attn_backward_bf16(const void* X, int B, int S, int h, int H, int d, int t, const tp_shard* Wqkv,
+                             const void* const* bqkv, const tp_shard* Wo, const void* dY, const void* dX_add,
+                             int causal, void* dX, float* dWqkv, float* dbqkv, float* dWo, float* dbo, void* ws,
+                             cudaStream_t stream) {
+  const int64_t M = static_cast<int64_t>(B) * S;
+  const int Hg = H / t;
+  const int64_t n = static_cast<int64_t>(Hg) * d;   // one group's columns of O / dO
+  const int64_t ncol = 3 * n;                       // one group's columns of QKV / dQKV
+  const int64_t Hd = static_cast<int64_t>(H) * d;
+  const int64_t S_pad = attn_s_pad(S);
+  AttnBwdWs w = attn_bwd_ws_layout(ws, B, S, H, d);
+  uint32_t* status = device_status_ptr();
+  const uint64_t lim = wait_limit_ns();
+  const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(d));
+  // 1. recompute Q, K, V (the forward's QKV projection)
+  {
+    GemmArgs a;
+    memset(&a, 0, sizeof(a));
+    TP_TRY(make_tmap_2d(&a.tmA, X, 0, h, M, static_cast<uint64_t>(h) * 2, 64, GEMM_BM));
+    for (int i = 0; i < t; ++i) TP_TRY(make_tmap_mn(&a.tmB[i], Wqkv[i].ptr, 0, ncol, h, Wqkv[i].ld * 2));
+    a.M = static_cast<int>(M); a.N = static_cast<int>(ncol); a.Kg = h; a.G = t;
+    a.epi = EPI_QKV; a.act = ACT_NONE;
+    for (int i = 0; i < t; ++i) a.bias_g[i] = bqkv ? bqkv[i] : nullptr;
+    a.q = w.fwd.q; a.k = w.fwd.k; a.v = w.fwd.v; a.S = S; a.H = H; a.Hg = Hg; a.d = d;
+    a.status = status; a.wait_limit_ns = lim;
+    TP_TRY(launch_gemm(a, stream, "gemm_qkv"));
+  }
+  // 2. recompute O (bf16) and each softmax row's log2-sum-exp
+  {
+    AttnArgs a;
+    memset(&a, 0, sizeof(a));
+    TP_TRY(make_tmap_attn(&a.tmQ, w.fwd.q, B * H, S, d, 128));
+    TP_TRY(make_tmap_attn(&a.tmK, w.fwd.k, B * H, S, d, attention_kv_rows()));
+    TP_TRY(make_tmap_attn(&a.tmV, w.fwd.v, B * H, S, d, attention_kv_rows()));
+    a.O = w.fwd.o; a.o_f16 = 0;
+    a.B = B; a.S = S; a.H = H; a.d = d; a.causal = causal; a.head0 = 0;
+    a.scale_log2 = scale_log2;
+    a.lse = w.lse; a.lse_ld = static_cast<int>(S_pad);
+    a.status = status; a.wait_limit_ns = lim;
+    TP_TRY(launch_attention(a, stream));
+  }
+  // 3. dbo = column sums of dY
+  if (dbo) TP_TRY(launch_colsum(dY, M, h, h, w.colsum, dbo, stream));
+  // 4. dWo_i = O_i^T dY (rows i*n.. of dWo): the row-parallel projection's weight gradient
+  {
+    GemmArgs a;
+    memset(&a, 0, sizeof(a));
+    TP_TRY(make_tmap_mn(&a.tmA, w.fwd.o, 0, Hd, M, Hd * 2));
+    for (int i = 0; i < t; ++i) TP_TRY(make_tmap_mn(&a.tmB[i], dY, 0, h, M, h * 2));
+    a.M = static_cast<int>(n); a.N = h; a.Kg = static_cast<int>(M); a.G = t;
+    a.a_mn = 1; a.a_m_per_group = static_cast<int>(n);
+    a.epi = EPI_PARTIAL_F32;
+    a.out = dWo; a.ld_out = h; a.out_group_stride = n * h;
+    TP_TRY(make_tmap_out_f32_3d(&a.tmOut, dWo, h, n, t, h * 4, n * h * 4));
+    a.tma_store = 1;
+    a.status = status; a.wait_limit_ns = lim;
+    TP_TRY(launch_gemm(a, stream, "gemm_attn_bwd_dwo"));
+  }
+  // 5. dO_i = dY Wo_i^T (fp16): the row-parallel projection's input gradient, local to group i
+  {
+    GemmArgs a;
+    memset(&a, 0, sizeof(a));
+    TP_TRY(make_tmap_2d(&a.tmA, dY, 0, h, M, static_cast<uint64_t>(h) * 2, 64, GEMM_BM));
+    for (int i = 0; i < t; ++i) TP_TRY(make_tmap_2d(&a.tmB[i], Wo[i].ptr, 0, h, n, Wo[i].ld * 2, 64, 128));
+    TP_TRY(make_tmap_out(&a.tmOut, w.dO, 1, static_cast<uint64_t>(Hd), M, Hd * 2));
+    a.M = static_cast<int>(M); a.N = static_cast<int>(n); a.Kg = h; a.G = t;
+    a.b_kmajor = 1;
+    a.epi = EPI_ACT; a.act = ACT_NONE;
+    a.out = w.dO; a.ld_out = Hd; a.out_col_per_group = n; a.out_type = OUT_F16; a.tma_store = 1;
+    a.status = status; a.wait_limit_ns = lim;
+    TP_TRY(launch_gemm(a, stream, "gemm_attn_bwd_do"));
+  }
+  // 6. per-head attention gradients into dQKV
+  {
+    AttnBwdArgs a;
+    memset(&a, 0, sizeof(a));
+    TP_TRY(make_tmap_attn(&a.tmQ, w.fwd.q, B * H, S, d, 128));
+    TP_TRY(make_tmap_attn(&a.tmK, w.fwd.k, B * H, S, d, 128));
+    TP_TRY(make_tmap_attn(&a.tmV, w.fwd.v, B * H, S, d, 128));
+    TP_TRY(make_tmap_rows_by_head(&a.tmdO, w.dO, B, S, H, d));
+    a.lse = w.lse; a.Dv = w.Dv; a.dqkv = w.dqkv; a.ld_dqkv = 3 * Hd;
+    a.B = B; a.S = S; a.H = H; a.Hg = Hg; a.head0 = 0; a.causal = causal; a.S_pad = static_cast<int>(S_pad);
+    a.scale_log2 = scale_log2; a.scale = 1.f / sqrtf(static_cast<float>(d));
+    a.status = status; a.wait_limit_ns = lim;
+    TP_TRY(launch_attention_backward(a, w.dO, w.fwd.o, 0, stream));
+  }
+  // 7. dWqkv_i = X^T dQKV_i (columns i*3n.. of dWqkv): the column-parallel weight gradient
+  {
+    GemmArgs a;
+    memset(&a, 0, sizeof(a));
+    TP_TRY(make_tmap_mn(&a.tmA, X, 0, h, M, static_cast<uint64_t>(h) * 2));
+    for (int i = 0; i < t; ++i) TP_TRY(make_tmap_mn(&a.tmB[i], w.dqkv + i * ncol, 0, ncol, M, 3 * Hd * 2));
+    a.M = h; a.N = static_cast<int>(ncol); a.Kg = static_cast<int>(M); a.G = t;
+    a.a_mn = 1; a.a_m_per_group = 0;
+    a.epi = EPI_PARTIAL_F32;
+    a.out = dWqkv; a.ld_out = 3 * Hd; a.out_group_stride = ncol;
+    TP_TRY(make_tmap_out_f32_3d(&a.tmOut, dWqkv, ncol, h, t, 3 * Hd * 4, ncol * 4));
+    a.tma_store = 1;
+    a.status = status; a.wait_limit_ns = lim;
+    TP_TRY(launch_gemm(a, stream, "gemm_attn_bwd_dwqkv"));
+  }
+  // 8. dbqkv = column sums of dQKV
+  if (dbqkv) TP_TRY(launch_colsum(w.dqkv, M, 3 * Hd, 3 * Hd, w.colsum, dbqkv, stream));
+  // 9. dX = sum_i dQKV_i Wqkv_i^T (+ dX_add): the sum over head groups, in one accumulator
+  {
+    GemmArgs a;
+    memset(&a, 0, sizeof(a));
+    TP_TRY(make_tmap_2d(&a.tmA, w.dqkv, 0, 3 * Hd, M, 3 * Hd * 2, 64, GEMM_BM));
+    for (int i = 0; i < t; ++i) TP_TRY(make_tmap_2d(&a.tmB[i], Wqkv[i].ptr, 0, ncol, h, Wqkv[i].ld * 2, 64, 128));
+    TP_TRY(make_tmap_out(&a.tmOut, dX, 0, static_cast<uint64_t>(h), M, h * 2));
+    a.M = static_cast<int>(M); a.N = h; a.Kg = static_cast<int>(ncol); a.G = t;
+    a.concat = 1; a.a_k_per_group = static_cast<int>(ncol); a.b_kmajor = 1;
+    a.epi = EPI_BIAS_RESID; a.bias = nullptr; a.resid = dX_add; a.ld_resid = h; a.resid_fp32 = 0;
+    a.out = dX; a.ld_out = h; a.out_type = OUT_BF16; a.tma_store = 1;
+    a.status = status; a.wait_limit_ns = lim;
+    TP_TRY(launch_gemm(a, stream, "gemm_attn_bwd_dx"));
+  }
+  return TP_OK;
+}
+
 tp_status validate_attn(const void* X, int B, int S, int h, int H, int d, int t, const tp_shard* Wqkv,
                         const void* const* bqkv, const tp_shard* Wo, const void* bo, const void* residual,
                         void* out, tp_reduce_mode mode, void* ws, size_t ws_bytes) {
@@ -816,6 +992,52 @@ tp_status tp_attn_forward(const void* X, int B, int S, int h, int heads, int d, 
                    static_cast<cudaStream_t>(stream));
 }
 
+size_t tp_attn_backward_workspace_bytes(int B, int S, int h, int heads, int d, int t) {
+  if (B <= 0 || S <= 0 || h <= 0 || heads <= 0 || d <= 0 || t < 1) return 0;
+  return attn_bwd_ws_bytes(B, S, h, heads, d);
+}
+
+tp_status tp_attn_backward(const void* X, int B, int S, int h, int heads, int d, int t, const tp_shard* Wqkv,
+                           const void* const* bqkv, const tp_shard* Wo, const void* dY, const void* dX_add,
+                           int causal, void* dX, float* dWqkv, float* dbqkv, float* dWo, float* dbo, void* ws,
+                           size_t ws_bytes, tp_stream_t stream) {
+  ApiRange range("tp_attn_backward");
+  TP_TRY(validate_attn_dims(B, S, h, heads, d, t));
+  const int64_t M = static_cast<int64_t>(B) * S;
+  const int64_t Hd = static_cast<int64_t>(heads) * d;
+  // with no tokens, X, dY and dX are never touched and may be NULL
+  TP_TRY(check_ptr(X, "X", M > 0));
+  TP_TRY(check_ptr(dY, "dY", M > 0));
+  TP_TRY(check_ptr(dX_add, "dX_add", false));
+  TP_TRY(check_ptr(dX, "dX", M > 0));
+  TP_TRY(check_ptr(dWqkv, "dWqkv", true));
+  TP_TRY(check_ptr(dWo, "dWo", true));
+  TP_TRY(check_ptr(dbqkv, "dbqkv", false));
+  TP_TRY(check_ptr(dbo, "dbo", false));
+  TP_TRY(check_shards(Wqkv, t, 3LL * (heads / t) * d, "Wqkv"));
+  TP_TRY(check_shards(Wo, t, h, "Wo"));
+  TP_TRY(check_bias_array(bqkv, t, "bqkv"));
+  if (is_f16(Wqkv) || is_f16(Wo)) return fail(TP_ERR_UNSUPPORTED, "the backward pass takes bf16 Wqkv and Wo");
+  if (M > 0 && (dX == X || dX == dY || dX == dX_add)) return fail(TP_ERR_INVALID_ARG, "dX aliases an input");
+  const size_t need = tp_attn_backward_workspace_bytes(B, S, h, heads, d, t);
+  if (need && (!ws || ws_bytes < need))
+    return fail(TP_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws ? ws_bytes : 0);
+  if (ws && (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN))
+    return fail(TP_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M == 0) {
+    // no tokens: every weight and bias gradient is zero
+    if (cudaMemsetAsync(dWqkv, 0, static_cast<size_t>(h) * 3 * Hd * 4, s) != cudaSuccess ||
+        cudaMemsetAsync(dWo, 0, static_cast<size_t>(Hd) * h * 4, s) != cudaSuccess ||
+        (dbqkv && cudaMemsetAsync(dbqkv, 0, static_cast<size_t>(3 * Hd) * 4, s) != cudaSuccess) ||
+        (dbo && cudaMemsetAsync(dbo, 0, static_cast<size_t>(h) * 4, s) != cudaSuccess))
+      return fail(TP_ERR_CUDA, "cudaMemsetAsync of the gradients failed");
+    return TP_OK;
+  }
+  return attn_backward_bf16(X, B, S, h, heads, d, t, Wqkv, bqkv, Wo, dY, dX_add, causal ? 1 : 0, dX, dWqkv, dbqkv,
+                            dWo, dbo, ws, s);
+}
+
 size_t tp_layer_workspace_bytes(int B, int S, int h, int heads, int d, int64_t f, int t, tp_reduce_mode mode) {
   if (B <= 0 || S <= 0 || h <= 0 || heads <= 0 || d <= 0 || f <= 0 || t < 1) return 0;
   const int64_t M = static_cast<int64_t>(B) * S;
@@ -929,6 +1151,7 @@ tp_status tp_get_device_status(tp_stream_t stream) {
     if (v & DEV_RANGE_QKV) where += " Q/K/V;";
     if (v & DEV_RANGE_ATTN_O) where += " attention output O;";
     if (v & DEV_RANGE_LAYERNORM) where += " LayerNorm output;";
+    if (v & DEV_RANGE_ATTN_GRAD) where += " attention backward P or dS;";
     return fail(TP_ERR_RANGE, "an fp16 intermediate exceeded 65504 in:%s", where.c_str());
   }
   return fail(TP_ERR_CUDA, "device status 0x%x", v);

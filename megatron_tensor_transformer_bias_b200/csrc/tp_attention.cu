@@ -362,6 +362,7 @@ __global__ void __launch_bounds__(THREADS, 2) tp_attention_kernel(const __grid_c
       if (__all_sync(0xffffffffu, mbar_wait_bounded(drain_bar, 0, a.wait_limit_ns, a.status, WAIT_SITE_ATTN))) {
         tc_fence_after();
         const float inv = 1.f / l_run;
+        if (a.lse && q < a.S) a.lse[static_cast<int64_t>(bh) * a.lse_ld + q] = m_ref + log2f(l_run);
         uint16_t* dst = static_cast<uint16_t*>(a.O) + (static_cast<int64_t>(b) * a.S + q) * (a.H * D) + head * D;
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
@@ -808,6 +809,7 @@ __global__ void __launch_bounds__(tt::THREADS, 1) tp_attention_tt_kernel(const _
       }
       tc_fence_after();
       const float inv = 1.f / l_run;
+      if (a.lse && q < a.S) a.lse[static_cast<int64_t>(it.bh) * a.lse_ld + q] = m_ref + log2f(l_run);
       uint16_t* dst =
           static_cast<uint16_t*>(a.O) + (static_cast<int64_t>(it.b) * a.S + q) * (a.H * D) + it.head * D;
       uint32_t o[4][32];

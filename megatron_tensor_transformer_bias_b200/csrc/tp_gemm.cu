@@ -1037,6 +1037,7 @@ static GemmKernel gemm_kernel_for(int epi, int opl, bool pair) {
   TP_GEMM_PICK(EPI_MUL_GRAD, OPL_B_KMAJOR)
   TP_GEMM_PICK(EPI_PARTIAL_F32, OPL_A_MN)
   TP_GEMM_PICK(EPI_BIAS_RESID, OPL_B_KMAJOR)
+  TP_GEMM_PICK(EPI_ACT, OPL_B_KMAJOR)
 #undef TP_GEMM_PICK
   return nullptr;
 }

@@ -20,7 +20,8 @@ enum : uint32_t {
   DEV_RANGE_QKV = 1u << 17,      // Q, K, V of the attention projection (always fp16)
   DEV_RANGE_ATTN_O = 1u << 18,   // attention output O, fp16
   DEV_RANGE_LAYERNORM = 1u << 19,  // LayerNorm output, fp16
-  DEV_RANGE_MASK = 0xFu << 16
+  DEV_RANGE_ATTN_GRAD = 1u << 20,  // attention backward: P^T, dS (fp16 tensor-memory operands)
+  DEV_RANGE_MASK = 0x1Fu << 16
 };
 constexpr float FP16_MAX = 65504.0f;
 enum : uint32_t {
@@ -108,6 +109,27 @@ struct AttnArgs {
   int B, S, H, d, causal;
   int head0;         // first head handled (head-group offset)
   float scale_log2;  // log2(e) / sqrt(d)
+  // Optional: per-row log2-sum-exp of the scaled scores, lse[(b*H + head) * lse_ld + s]
+  // (rows s < S only), so that exp2(s * scale_log2 - lse) is the softmax row.
+  float* lse;
+  int lse_ld;
+  uint32_t* status;
+  uint64_t wait_limit_ns;
+};
+
+// Attention backward (tp_attention_bwd.cu).  Q, K, V [B*H][S][d] fp16 with boxes of 128
+// rows; dO [B*S, H*d] fp16 as a 4-D map (d, H, S, B), box {64, 1, 128, 1}; lse and Dv
+// [B*H][S_pad] fp32 (S_pad = S rounded up to 128); dqkv [B*S, ld_dqkv] bf16, head group
+// g's columns [g*3*Hg*d, ...) = [dQ heads | dK heads | dV heads].
+struct AttnBwdArgs {
+  CUtensorMap tmQ, tmK, tmV, tmdO;
+  float* lse;
+  float* Dv;
+  uint16_t* dqkv;
+  int64_t ld_dqkv;
+  int B, S, H, Hg, head0, causal, S_pad;
+  float scale_log2;  // log2(e) / sqrt(d)
+  float scale;       // 1 / sqrt(d)
   uint32_t* status;
   uint64_t wait_limit_ns;
 };
@@ -136,6 +158,9 @@ tp_status launch_gemm(const GemmArgs& a, cudaStream_t stream, const char* name);
 tp_status launch_attention(const AttnArgs& a, cudaStream_t stream);
 // Rows of the K and V tensor-map boxes: the key-block size of the attention kernel in use.
 int attention_kv_rows();
+// D = rowsum(dO * O) (and the padding rows of D / lse), then dK, dV and dQ into a.dqkv.
+tp_status launch_attention_backward(const AttnBwdArgs& a, const uint16_t* dO, const uint16_t* O, int o_f16,
+                                    cudaStream_t stream);
 tp_status launch_reduce_partials(const float* P, int t, int64_t M, int64_t h, const void* bias, int bias_fp32,
                                  const void* resid, int resid_fp32, void* out, int out_fp32,
                                  cudaStream_t stream);

@@ -58,6 +58,9 @@ _SIGS = {
     "tp_attn_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32, _i32]),
     "tp_attn_forward": (_i32, [_vp, _i32, _i32, _i32, _i32, _i32, _i32, _SP, _VPP, _SP, _vp, _vp, _i32, _vp, _i32,
                                _vp, _sz, _vp]),
+    "tp_attn_backward_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32]),
+    "tp_attn_backward": (_i32, [_vp, _i32, _i32, _i32, _i32, _i32, _i32, _SP, _VPP, _SP, _vp, _vp, _i32, _vp, _vp,
+                                _vp, _vp, _vp, _vp, _sz, _vp]),
     "tp_layer_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32, _i64, _i32, _i32]),
     "tp_layer_forward": (_i32, [_vp, _i32, _i32, _i32, _i32, _i32, _i64, _i32, _vp, _vp, _SP, _VPP, _SP, _vp, _vp,
                                 _vp, _SP, _VPP, _SP, _vp, _f32, _i32, _vp, _i32, _vp, _sz, _vp]),
@@ -277,6 +280,29 @@ def tp_attn_forward(X, B, S, heads, d, Wqkv, bqkv, Wo, bo, residual, out, causal
                                  _ptr(bo), _ptr(residual), 1 if causal else 0, _ptr(out), m, _ptr(ws), ws.numel(),
                                  _stream(stream)))
     return out
+
+
+def tp_attn_backward_workspace_bytes(B, S, h, heads, d, t) -> int:
+    return lib().tp_attn_backward_workspace_bytes(B, S, h, heads, d, t)
+
+
+def tp_attn_backward(X, B, S, heads, d, Wqkv, bqkv, Wo, dY, dX, dWqkv, dWo, dbqkv=None, dbo=None, dX_add=None,
+                     causal=True, ws=None, stream=None):
+    """Gradients of the attention sub-layer (bf16): dX [B*S,h] bf16, dWqkv [h, 3*heads*d] fp32
+    (group i's [Q|K|V] column block i), dWo [heads*d, h] fp32, dbqkv [3*heads*d] and dbo [h]
+    fp32 (optional), for the upstream gradient dY [B*S,h] bf16."""
+    for t_ in (X, dY, dX, dWqkv, dWo):
+        _dev(t_)
+    h = X.shape[1]
+    t = len(Wqkv)
+    if dWqkv.dtype != torch.float32 or dWo.dtype != torch.float32:
+        raise ValueError("weight gradients are fp32")
+    if ws is None:
+        ws = workspace(tp_attn_backward_workspace_bytes(B, S, h, heads, d, t), X.device)
+    _check(lib().tp_attn_backward(_ptr(X), B, S, h, heads, d, t, _shards(Wqkv), _ptr_array(bqkv), _shards(Wo),
+                                  _ptr(dY), _ptr(dX_add), 1 if causal else 0, _ptr(dX), _ptr(dWqkv), _ptr(dbqkv),
+                                  _ptr(dWo), _ptr(dbo), _ptr(ws), ws.numel(), _stream(stream)))
+    return dX, dWqkv, dWo, dbqkv, dbo
 
 
 def tp_layer_workspace_bytes(B, S, h, heads, d, f, t, mode=TP_REDUCE_FUSED) -> int:

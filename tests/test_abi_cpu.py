@@ -192,3 +192,32 @@ def test_backward_validation(L):
     w2[0].dtype = w2[1].dtype = tb.TP_FP16
     assert call(W2=w2) == tb.TP_ERR_UNSUPPORTED and "bf16" in tb.last_error()
     assert call() == tb.TP_ERR_WORKSPACE and "workspace" in tb.last_error()
+
+
+def test_attn_backward_workspace_and_validation(L):
+    B, S, h, H, d, t = 2, 2048, 4096, 32, 128, 4
+    q = B * S * H * d * 2
+    vec = B * H * 2048 * 4
+    colsum = (B * S + 127) // 128 * (3 * H * d) * 4
+    assert tb.tp_attn_backward_workspace_bytes(B, S, h, H, d, t) == 8 * q + 2 * vec + colsum
+    assert tb.tp_attn_backward_workspace_bytes(0, S, h, H, d, t) == 0
+    # S not a multiple of 128: the row vectors are padded to whole 128-query blocks
+    assert tb.tp_attn_backward_workspace_bytes(1, 200, 256, 2, d, 1) >= 8 * (200 * 2 * d * 2) + 2 * 2 * 256 * 4
+
+    Bs, Ss, hs, Hs, ts = 1, 128, 256, 2, 2
+    n = (Hs // ts) * d
+
+    def call(**k):
+        return L.tp_attn_backward(k.get("X", FAKE), Bs, Ss, hs, Hs, k.get("d", d), ts, k.get("Wqkv", _sh(ts, 3 * n)),
+                                  None, k.get("Wo", _sh(ts, hs)), k.get("dY", FAKE + 8192), None, 1,
+                                  k.get("dX", FAKE + 4096), k.get("dWqkv", FAKE + 16384), None,
+                                  k.get("dWo", FAKE + 32768), None, k.get("ws", FAKE), 0, None)
+    assert call(dY=None) == tb.TP_ERR_INVALID_ARG and "dY is NULL" in tb.last_error()
+    assert call(dWqkv=None) == tb.TP_ERR_INVALID_ARG and "dWqkv is NULL" in tb.last_error()
+    assert call(dWo=None) == tb.TP_ERR_INVALID_ARG and "dWo is NULL" in tb.last_error()
+    assert call(dX=FAKE) == tb.TP_ERR_INVALID_ARG and "alias" in tb.last_error()
+    assert call(d=64) == tb.TP_ERR_UNSUPPORTED and "d=64" in tb.last_error()
+    wo = _sh(ts, hs)
+    wo[0].dtype = wo[1].dtype = tb.TP_FP16
+    assert call(Wo=wo) == tb.TP_ERR_UNSUPPORTED and "bf16" in tb.last_error()
+    assert call() == tb.TP_ERR_WORKSPACE and "workspace" in tb.last_error()

@@ -77,8 +77,9 @@ def test_reference_arm_tiny_fp32_and_workload_order(capsys, monkeypatch):
     class A:
         workload, impl, mode, t, h = "all", "ours", "fused", 4, "22528"
     names = [w.name for w in bench.make_workloads(A)]
-    assert names[-1] == "ffn_bf16_M2048_h4096_f16384_t4" and len(names) == len(set(names)) == 8
+    assert names[-1] == "ffn_bf16_M2048_h4096_f16384_t4" and len(names) == len(set(names)) == 9
     assert "ffn_bwd_bf16_M2048_h4096_f16384_t4" in names
+    assert "attn_bwd_bf16_B2_S2048_h4096_H32_d128_t4_causal" in names
     A.impl = "reference"
     assert bench.make_workloads(A)[-1].headline
 
@@ -96,3 +97,17 @@ def test_kernel_source_hash_ignores_comments_only():
     assert bench._kernel_sha("attention") != bench._kernel_sha("gemm_row_fused_reduce")
     assert bench._kernel_sha("gemm_column_act") == bench._kernel_sha("gemm_row_fused_reduce")
     assert bench._kernel_sha("not_a_kernel") == bench._csrc_sha()
+
+
+def test_reference_arm_attention_backward(capsys, monkeypatch):
+    """The attention backward's reference line: the oracle on one head over one sequence
+    per step, credited 1/(B*H) of the workload's FLOPs."""
+    import json
+    import sys
+    import bench
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--workload", "attn_bwd", "--steps", "1",
+                                      "--warmup", "3"])
+    bench.main()
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["config"]["workload"] == "attn_bwd_bf16_B2_S2048_h4096_H32_d128_t4_causal"
+    assert line["value"] > 0 and "one head over one sequence" in line["cpu_baseline"]["sample"]
