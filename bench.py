@@ -89,6 +89,13 @@ KERNEL_SOURCES = {
     "gemm_bwd_dw1": ["tp_gemm.cu"] + _SHARED_SOURCES,
     "gemm_bwd_dx": ["tp_gemm.cu"] + _SHARED_SOURCES,
     "colsum": ["tp_simt.cu"] + _SHARED_SOURCES,
+    "gemm_attn_bwd_dwo": ["tp_gemm.cu"] + _SHARED_SOURCES,
+    "gemm_attn_bwd_do": ["tp_gemm.cu"] + _SHARED_SOURCES,
+    "gemm_attn_bwd_dwqkv": ["tp_gemm.cu"] + _SHARED_SOURCES,
+    "gemm_attn_bwd_dx": ["tp_gemm.cu"] + _SHARED_SOURCES,
+    "attn_bwd_rowdot": ["tp_attention_bwd.cu"] + _SHARED_SOURCES,
+    "attn_bwd_dkdv": ["tp_attention_bwd.cu"] + _SHARED_SOURCES,
+    "attn_bwd_dq": ["tp_attention_bwd.cu"] + _SHARED_SOURCES,
 }
 
 
