@@ -237,16 +237,16 @@ tp_status make_tmap_attn(CUtensorMap* map, const void* base, int BH, int S, int 
                            static_cast<uint64_t>(S) * d * 2, 64, box_rows);
 }
 
-// [B*S, H*d] fp16 (token rows, head-major columns) seen as (d, H, S, B): box {64, 1, 128, 1}
-// is 128 rows of one head's 64 columns, the same shared-memory tile as make_tmap_attn's.
-tp_status make_tmap_rows_by_head(CUtensorMap* map, const void* base, int B, int S, int H, int d) {
+// [B*S, H*d] fp16 (token rows, head-major columns) seen as (d, H, S, B): box {64, 1, rows, 1}
+// is `rows` rows of one head's 64 columns, the same shared-memory tile as make_tmap_attn's.
+tp_status make_tmap_rows_by_head(CUtensorMap* map, const void* base, int B, int S, int H, int d, uint32_t box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(S),
                         static_cast<cuuint64_t>(B)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2,
                            static_cast<cuuint64_t>(S) * H * d * 2};
-  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t box[4] = {64, 1, box_rows, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -774,7 +774,11 @@ tp_status attn_backward_bf16(const void* X, int B, int S, int h, int H, int d, i
     TP_TRY(make_tmap_attn(&a.tmQ, w.fwd.q, B * H, S, d, 128));
     TP_TRY(make_tmap_attn(&a.tmK, w.fwd.k, B * H, S, d, 128));
     TP_TRY(make_tmap_attn(&a.tmV, w.fwd.v, B * H, S, d, 128));
-    TP_TRY(make_tmap_rows_by_head(&a.tmdO, w.dO, B, S, H, d));
+    TP_TRY(make_tmap_rows_by_head(&a.tmdO, w.dO, B, S, H, d, 128));
+    TP_TRY(make_tmap_attn(&a.tmQs, w.fwd.q, B * H, S, d, 64));
+    TP_TRY(make_tmap_attn(&a.tmKs, w.fwd.k, B * H, S, d, 64));
+    TP_TRY(make_tmap_attn(&a.tmVs, w.fwd.v, B * H, S, d, 64));
+    TP_TRY(make_tmap_rows_by_head(&a.tmdOs, w.dO, B, S, H, d, 64));
     a.lse = w.lse; a.Dv = w.Dv; a.dqkv = w.dqkv; a.ld_dqkv = 3 * Hd;
     a.B = B; a.S = S; a.H = H; a.Hg = Hg; a.head0 = 0; a.causal = causal; a.S_pad = static_cast<int>(S_pad);
     a.scale_log2 = scale_log2; a.scale = 1.f / sqrtf(static_cast<float>(d));

@@ -11,16 +11,19 @@
 //     dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),
 //     dQ = dS K / sqrt(d),  dK = dS^T Q / sqrt(d).
 // rowsum(P * dP) = rowsum(dO * O) because O = P V, so D is the softmax Jacobian's
-// row correction.  Two kernels, each one 128-row block per CTA and no atomics (the
-// sums over blocks run in one TMEM accumulator, in block order):
+// row correction.  Two kernels, each one resident 128-row block per CTA and no
+// atomics (the sums run in one TMEM accumulator, in sub-block order):
 //  * tp_attn_bwd_dkdv_kernel: one CTA per (128 keys, head, batch).  It keeps K_j and
-//    V_j in shared memory and walks the query blocks that see them:
-//    S^T = K_j Q_i^T and dP^T = V_j dO_i^T into TMEM; the compute warps (one key row
-//    per thread) form P^T and dS^T in fp16 over them; then dV += P^T dO_i and
-//    dK += dS^T Q_i read those from TMEM.
+//    V_j in shared memory and streams the 64-query sub-blocks that see them:
+//    S^T = K_j Q_n^T and dP^T = V_j dO_n^T into TMEM; the compute warps (one key row
+//    per thread) form P^T and dS^T in fp16 over them; then dV += P^T dO_n and
+//    dK += dS^T Q_n read those from TMEM.
 //  * tp_attn_bwd_dq_kernel: one CTA per (128 queries, head, batch).  It keeps Q_i
-//    and dO_i and walks the key blocks the queries see: S = Q_i K_j^T and
-//    dP = dO_i V_j^T; dS (one query row per thread); dQ += dS K_j.
+//    and dO_i and streams the 64-key sub-blocks the queries see: S = Q_i K_n^T and
+//    dP = dO_i V_n^T; dS (one query row per thread); dQ += dS K_n.
+// The score tiles are double-buffered in TMEM: the tensor core computes sub-block
+// n+1's S and dP while the compute warps work on sub-block n, and the gradient MMAs
+// of n run right after its compute.
 // Each recomputes S (the forward's scores) instead of storing them.  Q, K, V are
 // [B*H][S][d] fp16 (the forward's workspace), dO is [B*S, H*d] fp16 (read through a
 // 4-D tensor map), LSE2 and D are [B*H][S_pad] fp32 with S_pad a multiple of 128 and
@@ -36,22 +39,29 @@ namespace tpb {
 
 namespace {
 
-constexpr int BR = 128;                      // rows per block (queries or keys)
+constexpr int BR = 128;                      // resident rows per CTA (keys or queries)
+constexpr int BS = 64;                       // streamed rows per sub-block
 constexpr int D = 128;                       // head dim
-constexpr int HALF = BR * 64 * 2;            // [128 rows x 64 d] fp16, 128-byte swizzle: 16 KB
-constexpr int TILE = 2 * HALF;               // 32 KB
+constexpr int HALF_R = BR * 64 * 2;          // [128 rows x 64 d] fp16, 128-byte swizzle: 16 KB
+constexpr int TILE_R = 2 * HALF_R;           // 32 KB
+constexpr int HALF_S = BS * 64 * 2;          // [64 rows x 64 d]: 8 KB
+constexpr int TILE_S = 2 * HALF_S;           // 16 KB
+constexpr int NST = 4;                       // shared-memory stages of streamed sub-blocks
 constexpr int THREADS = 192;                 // warp 0 TMA, warp 1 MMA, warps 2..5 compute
 constexpr int COMPUTE_THREADS = 128;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t IDESC_SS = idesc_f16_f32(BR, BR, 0, 0);   // both operands K-major (N = rows)
+constexpr uint32_t IDESC_SS = idesc_f16_f32(BR, BS, 0, 0);   // resident x streamed^T, both K-major
 constexpr uint32_t IDESC_TS = idesc_f16_f32(BR, D, 0, 1);    // A from TMEM, B N-major (N = d)
 
-// dK/dV kernel shared memory: K, V resident; two stages of (Q, dO, LSE2 and D of 128 queries)
-constexpr int VEC_BYTES = BR * 4;
-constexpr int KV_STAGE_BYTES = 2 * TILE + 2 * VEC_BYTES;
-constexpr int DKDV_SMEM = 1024 + 2 * TILE + 2 * KV_STAGE_BYTES + 256;
-// dQ kernel shared memory: Q, dO resident; two stages of (K, V)
-constexpr int DQ_SMEM = 1024 + 2 * TILE + 2 * (2 * TILE) + 256;
+// dK/dV: stage = Q_n, dO_n, LSE2 and D of 64 queries (padded to 1 KB)
+constexpr int VEC_BYTES = BS * 4;
+constexpr int STAGE_KV = ((2 * TILE_S + 2 * VEC_BYTES + 1023) / 1024) * 1024;
+constexpr int DKDV_SMEM = 1024 + 2 * TILE_R + NST * STAGE_KV + 256;
+// dQ: stage = K_n, V_n of 64 keys
+constexpr int STAGE_Q = 2 * TILE_S;
+constexpr int DQ_SMEM = 1024 + 2 * TILE_R + NST * STAGE_Q + 256;
+// TMEM: score buffer b at b*128 (64 columns), its dP at b*128 + 64; accumulators at 256 (and 384)
+constexpr uint32_t T_ACC0 = 256, T_ACC1 = 384;
 
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                        uint32_t accumulate) {
@@ -94,26 +104,27 @@ __device__ __forceinline__ float ex2f(float x) {
   return y;
 }
 
-// Descriptor of a [128 rows x 128 d] K-major tile (two 64-d halves), K step kk of 16.
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int kk) {
-  return smem_desc_sw128(base + (kk >> 2) * HALF + (kk & 3) * 32, 16, 1024);
+// K-major tile (two 64-d halves of `half` bytes each), K step kk of 16 along d.
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int kk, uint32_t half) {
+  return smem_desc_sw128(base + (kk >> 2) * half + (kk & 3) * 32, 16, 1024);
 }
-// Descriptor of the same tile read N-major (N = d), K step kk of 16 rows.
+// A streamed [64 rows x 128 d] tile read N-major (N = d), K step kk of 16 rows.
 __device__ __forceinline__ uint64_t nmajor_desc(uint32_t base, int kk) {
-  return smem_desc_sw128(base + kk * 16 * 128, HALF, 1024);
+  return smem_desc_sw128(base + kk * 16 * 128, HALF_S, 1024);
 }
 
-// Issue one 128 x 128 x 128 product with both operands K-major in shared memory.
+// D[128 x 64] = A[resident 128 x d] * B[streamed 64 x d]^T, both K-major in shared memory.
 __device__ __forceinline__ void mma_ss_tile(uint32_t d_tmem, uint32_t a_base, uint32_t b_base) {
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk)
-    mma_bf16_ss(d_tmem, kmajor_desc(a_base, kk), kmajor_desc(b_base, kk), IDESC_SS, kk > 0 ? 1u : 0u);
+    mma_bf16_ss(d_tmem, kmajor_desc(a_base, kk, HALF_R), kmajor_desc(b_base, kk, HALF_S), IDESC_SS,
+                kk > 0 ? 1u : 0u);
 }
 
-// D += A[tmem, 128 x 128 fp16] * B[smem, 128 rows x 128 d, read N-major].
+// D[128 x d] (+)= A[tmem, 128 x 64 fp16] * B[streamed 64 x d, read N-major].
 __device__ __forceinline__ void mma_ts_tile(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base, bool accumulate) {
 #pragma unroll
-  for (int kk = 0; kk < BR / 16; ++kk)
+  for (int kk = 0; kk < BS / 16; ++kk)
     mma_ts(d_tmem, a_tmem + static_cast<uint32_t>(kk * 8), nmajor_desc(b_base, kk), IDESC_TS,
            (accumulate || kk > 0) ? 1u : 0u);
 }
@@ -135,53 +146,82 @@ __device__ __forceinline__ void store_row_bf16(uint16_t* dst, const uint32_t (&v
   }
 }
 
+// The MMA thread's schedule, shared by both kernels: S and dP of sub-blocks 0 and 1 into
+// the two score buffers, then per sub-block n: (wait for its P / dS) the gradient MMAs of
+// n, release its stage, and S and dP of n + 2 into the buffer n just freed.
+template <typename SS, typename TS>
+__device__ __forceinline__ bool mma_schedule(int N, uint64_t* st_full, uint64_t* st_empty, uint64_t* s_full,
+                                             uint64_t* p_full, const AttnBwdArgs& a, SS issue_ss, TS issue_ts) {
+  for (int n = 0; n < N && n < 2; ++n) {
+    if (!mbar_wait_bounded(&st_full[n % NST], (n / NST) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN))
+      return false;
+    tc_fence_after();
+    issue_ss(n);
+    mma_commit(&s_full[n & 1]);
+  }
+  for (int n = 0; n < N; ++n) {
+    const int b = n & 1;
+    if (!mbar_wait_bounded(&p_full[b], (n >> 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN)) return false;
+    tc_fence_after();
+    issue_ts(n);
+    mma_commit(&st_empty[n % NST]);
+    const int m = n + 2;
+    if (m < N) {
+      if (!mbar_wait_bounded(&st_full[m % NST], (m / NST) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN))
+        return false;
+      tc_fence_after();
+      issue_ss(m);
+      mma_commit(&s_full[b]);
+    }
+  }
+  return true;
+}
+
 // ------------------------------------------------------------------------------ D
-// D[bh][s] = sum_e dO[b*S+s][h*d+e] * O[b*S+s][h*d+e] (one warp per (row, head)), and the
-// padding rows s in [S, S_pad) of D and LSE2 set to (0, +inf).
+// D[bh][s] = sum_e dO[b*S+s][h*d+e] * O[b*S+s][h*d+e]: 16 threads per (row, head), 8 columns
+// (16 bytes) each; the padding rows s in [S, S_pad) of D and LSE2 set to (0, +inf).
 __global__ void __launch_bounds__(256) tp_attn_bwd_rowdot_kernel(const uint16_t* __restrict__ dO,
                                                                  const uint16_t* __restrict__ O, int o_f16,
                                                                  float* __restrict__ Dv, float* __restrict__ lse,
                                                                  int B, int S, int H, int S_pad) {
   pdl_wait();
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
-  const int lane = threadIdx.x % 32;
+  const int64_t item = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 16;
+  const int sub = threadIdx.x % 16;
   const int64_t total = static_cast<int64_t>(B) * H * S_pad;
-  if (warp < total) {
-    const int s = static_cast<int>(warp % S_pad);
-    const int64_t bh = warp / S_pad;
+  float acc = 0.f;
+  int s = 0;
+  if (item < total) {
+    s = static_cast<int>(item % S_pad);
+    const int64_t bh = item / S_pad;
     const int h = static_cast<int>(bh % H);
     const int b = static_cast<int>(bh / H);
-    if (s >= S) {
-      if (lane == 0) {
-        Dv[warp] = 0.f;
-        lse[warp] = INFINITY;
-      }
-    } else {
-      const int64_t off = (static_cast<int64_t>(b) * S + s) * (static_cast<int64_t>(H) * D) + h * D + lane * 4;
-      const uint2 g = *reinterpret_cast<const uint2*>(dO + off);
-      const uint2 o = *reinterpret_cast<const uint2*>(O + off);
-      const __half2* g2 = reinterpret_cast<const __half2*>(&g);
-      float acc = 0.f;
+    if (s < S) {
+      const int64_t off = (static_cast<int64_t>(b) * S + s) * (static_cast<int64_t>(H) * D) + h * D + sub * 8;
+      const uint4 g = *reinterpret_cast<const uint4*>(dO + off);
+      const uint4 o = *reinterpret_cast<const uint4*>(O + off);
+      const uint32_t gw[4] = {g.x, g.y, g.z, g.w}, ow[4] = {o.x, o.y, o.z, o.w};
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const float2 gf = __half22float2(g2[k]);
-        const uint32_t ow = k == 0 ? o.x : o.y;
+      for (int k = 0; k < 4; ++k) {
+        const float2 gf = __half22float2(*reinterpret_cast<const __half2*>(&gw[k]));
         float o0, o1;
         if (o_f16) {
-          const float2 of = __half22float2(*reinterpret_cast<const __half2*>(&ow));
+          const float2 of = __half22float2(*reinterpret_cast<const __half2*>(&ow[k]));
           o0 = of.x;
           o1 = of.y;
         } else {
-          o0 = __uint_as_float(ow << 16);
-          o1 = __uint_as_float(ow & 0xFFFF0000u);
+          o0 = __uint_as_float(ow[k] << 16);
+          o1 = __uint_as_float(ow[k] & 0xFFFF0000u);
         }
         acc = fmaf(gf.x, o0, acc);
         acc = fmaf(gf.y, o1, acc);
       }
-#pragma unroll
-      for (int m = 16; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
-      if (lane == 0) Dv[warp] = acc;
     }
+  }
+#pragma unroll
+  for (int m = 8; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+  if (item < total && sub == 0) {
+    Dv[item] = s < S ? acc : 0.f;
+    if (s >= S) lse[item] = INFINITY;
   }
   pdl_launch_dependents();
 }
@@ -192,37 +232,39 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attn_bwd_dkdv_kernel(const __gr
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sK = smem;
-  uint8_t* sV = sK + TILE;
-  uint8_t* sStage = sV + TILE;               // [2] x {Q, dO, LSE2[128], D[128]}
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sStage + 2 * KV_STAGE_BYTES);
-  uint64_t* kv_full = bars + 0;
-  uint64_t* st_full = bars + 1;              // [2]
-  uint64_t* st_empty = bars + 3;             // [2]
-  uint64_t* s_full = bars + 5;
-  uint64_t* p_full = bars + 6;
-  uint64_t* done_bar = bars + 7;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
+  uint8_t* sV = sK + TILE_R;
+  uint8_t* sStage = sV + TILE_R;             // [NST] x {Q_n, dO_n, LSE2[64], D[64]}
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sStage + NST * STAGE_KV);
+  uint64_t* res_full = bars + 0;
+  uint64_t* st_full = bars + 1;              // [NST]
+  uint64_t* st_empty = bars + 1 + NST;       // [NST]
+  uint64_t* s_full = bars + 1 + 2 * NST;     // [2] per score buffer
+  uint64_t* p_full = bars + 3 + 2 * NST;     // [2] per score buffer, 128 arrivals
+  uint64_t* done_bar = bars + 5 + 2 * NST;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6 + 2 * NST);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int kb = static_cast<int>(blockIdx.x);        // key block (causal: fewest query blocks last)
+  const int kb = static_cast<int>(blockIdx.x);        // key block (causal: most query sub-blocks first)
   const int head = a.head0 + static_cast<int>(blockIdx.y);
   const int b = blockIdx.z;
   const int bh = b * a.H + head;
   const int k0 = kb * BR;
-  const int nqb_all = (a.S + BR - 1) / BR;
-  const int qb_first = a.causal ? kb : 0;
-  const int nq = nqb_all - qb_first;                  // query blocks that see this key block
+  const int nsb_all = (a.S + BS - 1) / BS;
+  const int sb_first = a.causal ? k0 / BS : 0;        // the first query sub-block that sees these keys
+  const int N = nsb_all - sb_first;
 
   if (threadIdx.x == 0) {
-    mbar_init(kv_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    mbar_init(res_full, 1);
+    for (int i = 0; i < NST; ++i) {
       mbar_init(&st_full[i], 1);
       mbar_init(&st_empty[i], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(p_full, COMPUTE_THREADS);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], COMPUTE_THREADS);
+    }
     mbar_init(done_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -236,76 +278,62 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attn_bwd_dkdv_kernel(const __gr
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // TMEM: S^T [0,128) (P^T over its first 64 columns), dP^T [128,256) (dS^T likewise),
-  // dV [256,384), dK [384,512)
-  const uint32_t T_ST = 0, T_DPT = 128, T_DV = 256, T_DK = 384;
   pdl_wait();
 
   if (warp == 0) {
     if (lane == 0) {
-      tma_prefetch_desc(&a.tmQ);
       tma_prefetch_desc(&a.tmK);
       tma_prefetch_desc(&a.tmV);
-      tma_prefetch_desc(&a.tmdO);
-      mbar_arrive_expect_tx(kv_full, 2 * TILE);
-      load_3d(sK, &a.tmK, kv_full, 0, k0, bh);
-      load_3d(sK + HALF, &a.tmK, kv_full, 64, k0, bh);
-      load_3d(sV, &a.tmV, kv_full, 0, k0, bh);
-      load_3d(sV + HALF, &a.tmV, kv_full, 64, k0, bh);
+      tma_prefetch_desc(&a.tmQs);
+      tma_prefetch_desc(&a.tmdOs);
+      mbar_arrive_expect_tx(res_full, 2 * TILE_R);
+      load_3d(sK, &a.tmK, res_full, 0, k0, bh);
+      load_3d(sK + HALF_R, &a.tmK, res_full, 64, k0, bh);
+      load_3d(sV, &a.tmV, res_full, 0, k0, bh);
+      load_3d(sV + HALF_R, &a.tmV, res_full, 64, k0, bh);
       int issued = 0;
-      for (int n = 0; n < nq; ++n) {
+      for (int n = 0; n < N; ++n) {
         if (*abort_flag) break;
-        const int st = n & 1;
-        if (!mbar_wait_bounded(&st_empty[st], ((n >> 1) & 1) ^ 1u, a.wait_limit_ns, a.status, WAIT_SITE_ATTN)) {
+        const int st = n % NST;
+        if (!mbar_wait_bounded(&st_empty[st], ((n / NST) & 1) ^ 1u, a.wait_limit_ns, a.status, WAIT_SITE_ATTN)) {
           *abort_flag = 1;
           break;
         }
-        const int q0 = (qb_first + n) * BR;
-        uint8_t* stage = sStage + st * KV_STAGE_BYTES;
-        mbar_arrive_expect_tx(&st_full[st], 2 * TILE + 2 * VEC_BYTES);
-        load_3d(stage, &a.tmQ, &st_full[st], 0, q0, bh);
-        load_3d(stage + HALF, &a.tmQ, &st_full[st], 64, q0, bh);
-        load_4d(stage + TILE, &a.tmdO, &st_full[st], 0, head, q0, b);
-        load_4d(stage + TILE + HALF, &a.tmdO, &st_full[st], 64, head, q0, b);
-        load_bulk(stage + 2 * TILE, a.lse + static_cast<int64_t>(bh) * a.S_pad + q0, VEC_BYTES, &st_full[st]);
-        load_bulk(stage + 2 * TILE + VEC_BYTES, a.Dv + static_cast<int64_t>(bh) * a.S_pad + q0, VEC_BYTES,
+        const int q0 = (sb_first + n) * BS;
+        uint8_t* stage = sStage + st * STAGE_KV;
+        mbar_arrive_expect_tx(&st_full[st], 2 * TILE_S + 2 * VEC_BYTES);
+        load_3d(stage, &a.tmQs, &st_full[st], 0, q0, bh);
+        load_3d(stage + HALF_S, &a.tmQs, &st_full[st], 64, q0, bh);
+        load_4d(stage + TILE_S, &a.tmdOs, &st_full[st], 0, head, q0, b);
+        load_4d(stage + TILE_S + HALF_S, &a.tmdOs, &st_full[st], 64, head, q0, b);
+        load_bulk(stage + 2 * TILE_S, a.lse + static_cast<int64_t>(bh) * a.S_pad + q0, VEC_BYTES, &st_full[st]);
+        load_bulk(stage + 2 * TILE_S + VEC_BYTES, a.Dv + static_cast<int64_t>(bh) * a.S_pad + q0, VEC_BYTES,
                   &st_full[st]);
         ++issued;
       }
-      mbar_wait_bounded(kv_full, 0, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
-      for (int n = issued - 2 > 0 ? issued - 2 : 0; n < issued; ++n)
-        mbar_wait_bounded(&st_full[n & 1], (n >> 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
+      mbar_wait_bounded(res_full, 0, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
+      for (int n = issued - NST > 0 ? issued - NST : 0; n < issued; ++n)
+        mbar_wait_bounded(&st_full[n % NST], (n / NST) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t kA = smem_u32(sK), vA = smem_u32(sV);
-      bool ok = mbar_wait_bounded(kv_full, 0, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
-      for (int n = 0; n <= nq && ok; ++n) {
-        if (n >= 1) {
-          // dV += P^T dO_{n-1}, dK += dS^T Q_{n-1}; their stage is free afterwards
-          const int sp = (n - 1) & 1;
-          if (!mbar_wait_bounded(p_full, (n - 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t stp = smem_u32(sStage + sp * KV_STAGE_BYTES);
-          mma_ts_tile(tmem_base + T_DV, tmem_base + T_ST, stp + TILE, n > 1);
-          mma_ts_tile(tmem_base + T_DK, tmem_base + T_DPT, stp, n > 1);
-          mma_commit(&st_empty[sp]);
-        }
-        if (n < nq) {
-          const int st = n & 1;
-          if (!mbar_wait_bounded(&st_full[st], (n >> 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t sq = smem_u32(sStage + st * KV_STAGE_BYTES);
-          mma_ss_tile(tmem_base + T_ST, kA, sq);          // S^T = K Q^T
-          mma_ss_tile(tmem_base + T_DPT, vA, sq + TILE);  // dP^T = V dO^T
-          mma_commit(s_full);
-        }
+      bool ok = mbar_wait_bounded(res_full, 0, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
+      if (ok) {
+        ok = mma_schedule(
+            N, st_full, st_empty, s_full, p_full, a,
+            [&](int n) {  // S^T = K Q_n^T, dP^T = V dO_n^T into buffer n & 1
+              const uint32_t st = smem_u32(sStage + (n % NST) * STAGE_KV);
+              const uint32_t buf = tmem_base + static_cast<uint32_t>((n & 1) * 128);
+              mma_ss_tile(buf, kA, st);
+              mma_ss_tile(buf + 64, vA, st + TILE_S);
+            },
+            [&](int n) {  // dV += P^T dO_n, dK += dS^T Q_n
+              const uint32_t st = smem_u32(sStage + (n % NST) * STAGE_KV);
+              const uint32_t buf = tmem_base + static_cast<uint32_t>((n & 1) * 128);
+              mma_ts_tile(tmem_base + T_ACC0, buf, st + TILE_S, n > 0);
+              mma_ts_tile(tmem_base + T_ACC1, buf + 64, st, n > 0);
+            });
       }
       if (!ok) *abort_flag = 1;
       mma_commit(done_bar);
@@ -319,52 +347,50 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attn_bwd_dkdv_kernel(const __gr
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const float sl2 = a.scale_log2;
     bool ok = true;
-    for (int n = 0; n < nq && ok; ++n) {
+    for (int n = 0; n < N && ok; ++n) {
+      const int bsel = n & 1;
       if (!__all_sync(0xffffffffu,
-                      mbar_wait_bounded(s_full, n & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN))) {
+                      mbar_wait_bounded(&s_full[bsel], (n >> 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int q0 = (qb_first + n) * BR;
-      const float* vec = reinterpret_cast<const float*>(sStage + (n & 1) * KV_STAGE_BYTES + 2 * TILE);
-      const bool diag = a.causal && q0 == k0;       // the only block with keys after queries
+      const int q0 = (sb_first + n) * BS;
+      const float* vec = reinterpret_cast<const float*>(sStage + (n % NST) * STAGE_KV + 2 * TILE_S);
+      const bool diag = a.causal && q0 < k0 + BR;     // sub-blocks with keys after some queries
+      const uint32_t buf = tmem_base + lane_off + static_cast<uint32_t>(bsel * 128);
+      uint32_t sv[2][32], gv[2][32];
+      tmem_ld_32x32b_x32(buf, sv[0]);
+      tmem_ld_32x32b_x32(buf + 32, sv[1]);
+      tmem_ld_32x32b_x32(buf + 64, gv[0]);
+      tmem_ld_32x32b_x32(buf + 96, gv[1]);
+      tmem_ld_wait();
+      uint32_t pk[32], dk[32];
       float gmax = 0.f;
-#pragma unroll 1
-      for (int p = 0; p < 2; ++p) {
-        uint32_t sv[2][32], gv[2][32];
-        tmem_ld_32x32b_x32(tmem_base + lane_off + T_ST + p * 64, sv[0]);
-        tmem_ld_32x32b_x32(tmem_base + lane_off + T_ST + p * 64 + 32, sv[1]);
-        tmem_ld_32x32b_x32(tmem_base + lane_off + T_DPT + p * 64, gv[0]);
-        tmem_ld_32x32b_x32(tmem_base + lane_off + T_DPT + p * 64 + 32, gv[1]);
-        tmem_ld_wait();
-        uint32_t pk[32], dk[32];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < 2; ++c) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int j0 = p * 64 + c * 32 + 2 * i;   // query column within the block
-            float pr[2], ds[2];
+        for (int i = 0; i < 16; ++i) {
+          float pr[2], ds[2];
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int j = j0 + e;
-              float pv = ex2f(__uint_as_float(sv[c][2 * i + e]) * sl2 - vec[j]);
-              if (diag && k > q0 + j) pv = 0.f;
-              pr[e] = pv;
-              ds[e] = pv * (__uint_as_float(gv[c][2 * i + e]) - vec[BR + j]);
-              gmax = fmaxf(gmax, fabsf(ds[e]));
-            }
-            pk[c * 16 + i] = pack_f16x2(pr[0], pr[1]);
-            dk[c * 16 + i] = pack_f16x2(ds[0], ds[1]);
+          for (int e = 0; e < 2; ++e) {
+            const int j = c * 32 + 2 * i + e;   // query within the sub-block
+            float pv = ex2f(__uint_as_float(sv[c][2 * i + e]) * sl2 - vec[j]);
+            if (diag && k > q0 + j) pv = 0.f;
+            pr[e] = pv;
+            ds[e] = pv * (__uint_as_float(gv[c][2 * i + e]) - vec[BS + j]);
+            gmax = fmaxf(gmax, fabsf(ds[e]));
           }
+          pk[c * 16 + i] = pack_f16x2(pr[0], pr[1]);
+          dk[c * 16 + i] = pack_f16x2(ds[0], ds[1]);
         }
-        tmem_st_32x32b_x32(tmem_base + lane_off + T_ST + p * 32, pk);
-        tmem_st_32x32b_x32(tmem_base + lane_off + T_DPT + p * 32, dk);
       }
+      tmem_st_32x32b_x32(buf, pk);          // P^T over the scores' first 32 columns
+      tmem_st_32x32b_x32(buf + 64, dk);     // dS^T over dP^T's first 32 columns
       note_f16_range(a.status, gmax, DEV_RANGE_ATTN_GRAD);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[bsel]);
     }
     if (!ok) {
       *abort_flag = 1;
@@ -376,13 +402,13 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attn_bwd_dkdv_kernel(const __gr
       uint16_t* base = a.dqkv + row * a.ld_dqkv + static_cast<int64_t>(g) * 3 * a.Hg * D + hl * D;
       // dV (no scale), then dK (times 1/sqrt(d)); rows past the sequence are not written
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tmem_base + lane_off + T_DV + c * 32, v[c]);
+      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tmem_base + lane_off + T_ACC0 + c * 32, v[c]);
       tmem_ld_wait();
-      if (nq > 0 && k < a.S) store_row_bf16(base + 2 * a.Hg * D, v, 1.f);
+      if (N > 0 && k < a.S) store_row_bf16(base + 2 * a.Hg * D, v, 1.f);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tmem_base + lane_off + T_DK + c * 32, v[c]);
+      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tmem_base + lane_off + T_ACC1 + c * 32, v[c]);
       tmem_ld_wait();
-      if (nq > 0 && k < a.S) store_row_bf16(base + a.Hg * D, v, a.scale);
+      if (N > 0 && k < a.S) store_row_bf16(base + a.Hg * D, v, a.scale);
     } else {
       *abort_flag = 1;
     }
@@ -404,16 +430,16 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attn_bwd_dq_kernel(const __grid
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sQ = smem;
-  uint8_t* sdO = sQ + TILE;
-  uint8_t* sStage = sdO + TILE;              // [2] x {K, V}
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sStage + 4 * TILE);
-  uint64_t* q_full = bars + 0;
-  uint64_t* st_full = bars + 1;              // [2]
-  uint64_t* st_empty = bars + 3;             // [2]
-  uint64_t* s_full = bars + 5;
-  uint64_t* p_full = bars + 6;
-  uint64_t* done_bar = bars + 7;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
+  uint8_t* sdO = sQ + TILE_R;
+  uint8_t* sStage = sdO + TILE_R;            // [NST] x {K_n, V_n}
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sStage + NST * STAGE_Q);
+  uint64_t* res_full = bars + 0;
+  uint64_t* st_full = bars + 1;              // [NST]
+  uint64_t* st_empty = bars + 1 + NST;       // [NST]
+  uint64_t* s_full = bars + 1 + 2 * NST;     // [2]
+  uint64_t* p_full = bars + 3 + 2 * NST;     // [2], 128 arrivals
+  uint64_t* done_bar = bars + 5 + 2 * NST;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6 + 2 * NST);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32;
@@ -424,16 +450,19 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attn_bwd_dq_kernel(const __grid
   const int b = blockIdx.z;
   const int bh = b * a.H + head;
   const int q0 = qb * BR;
-  const int nk = a.causal ? qb + 1 : nqb;                   // key blocks these queries see
+  const int nsb_all = (a.S + BS - 1) / BS;
+  const int N = a.causal ? min(nsb_all, (q0 + BR - 1) / BS + 1) : nsb_all;   // key sub-blocks seen
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    mbar_init(res_full, 1);
+    for (int i = 0; i < NST; ++i) {
       mbar_init(&st_full[i], 1);
       mbar_init(&st_empty[i], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(p_full, COMPUTE_THREADS);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], COMPUTE_THREADS);
+    }
     mbar_init(done_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -447,70 +476,58 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attn_bwd_dq_kernel(const __grid
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // TMEM: S [0,128) (dS over its first 64 columns), dP [128,256), dQ [256,384)
-  const uint32_t T_S = 0, T_DP = 128, T_DQ = 256;
   pdl_wait();
 
   if (warp == 0) {
     if (lane == 0) {
       tma_prefetch_desc(&a.tmQ);
-      tma_prefetch_desc(&a.tmK);
-      tma_prefetch_desc(&a.tmV);
       tma_prefetch_desc(&a.tmdO);
-      mbar_arrive_expect_tx(q_full, 2 * TILE);
-      load_3d(sQ, &a.tmQ, q_full, 0, q0, bh);
-      load_3d(sQ + HALF, &a.tmQ, q_full, 64, q0, bh);
-      load_4d(sdO, &a.tmdO, q_full, 0, head, q0, b);
-      load_4d(sdO + HALF, &a.tmdO, q_full, 64, head, q0, b);
+      tma_prefetch_desc(&a.tmKs);
+      tma_prefetch_desc(&a.tmVs);
+      mbar_arrive_expect_tx(res_full, 2 * TILE_R);
+      load_3d(sQ, &a.tmQ, res_full, 0, q0, bh);
+      load_3d(sQ + HALF_R, &a.tmQ, res_full, 64, q0, bh);
+      load_4d(sdO, &a.tmdO, res_full, 0, head, q0, b);
+      load_4d(sdO + HALF_R, &a.tmdO, res_full, 64, head, q0, b);
       int issued = 0;
-      for (int n = 0; n < nk; ++n) {
+      for (int n = 0; n < N; ++n) {
         if (*abort_flag) break;
-        const int st = n & 1;
-        if (!mbar_wait_bounded(&st_empty[st], ((n >> 1) & 1) ^ 1u, a.wait_limit_ns, a.status, WAIT_SITE_ATTN)) {
+        const int st = n % NST;
+        if (!mbar_wait_bounded(&st_empty[st], ((n / NST) & 1) ^ 1u, a.wait_limit_ns, a.status, WAIT_SITE_ATTN)) {
           *abort_flag = 1;
           break;
         }
-        const int k0 = n * BR;
-        uint8_t* stage = sStage + st * 2 * TILE;
-        mbar_arrive_expect_tx(&st_full[st], 2 * TILE);
-        load_3d(stage, &a.tmK, &st_full[st], 0, k0, bh);
-        load_3d(stage + HALF, &a.tmK, &st_full[st], 64, k0, bh);
-        load_3d(stage + TILE, &a.tmV, &st_full[st], 0, k0, bh);
-        load_3d(stage + TILE + HALF, &a.tmV, &st_full[st], 64, k0, bh);
+        const int k0 = n * BS;
+        uint8_t* stage = sStage + st * STAGE_Q;
+        mbar_arrive_expect_tx(&st_full[st], 2 * TILE_S);
+        load_3d(stage, &a.tmKs, &st_full[st], 0, k0, bh);
+        load_3d(stage + HALF_S, &a.tmKs, &st_full[st], 64, k0, bh);
+        load_3d(stage + TILE_S, &a.tmVs, &st_full[st], 0, k0, bh);
+        load_3d(stage + TILE_S + HALF_S, &a.tmVs, &st_full[st], 64, k0, bh);
         ++issued;
       }
-      mbar_wait_bounded(q_full, 0, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
-      for (int n = issued - 2 > 0 ? issued - 2 : 0; n < issued; ++n)
-        mbar_wait_bounded(&st_full[n & 1], (n >> 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
+      mbar_wait_bounded(res_full, 0, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
+      for (int n = issued - NST > 0 ? issued - NST : 0; n < issued; ++n)
+        mbar_wait_bounded(&st_full[n % NST], (n / NST) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t qA = smem_u32(sQ), gA = smem_u32(sdO);
-      bool ok = mbar_wait_bounded(q_full, 0, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
-      for (int n = 0; n <= nk && ok; ++n) {
-        if (n >= 1) {
-          // dQ += dS K_{n-1}; its stage is free afterwards
-          const int sp = (n - 1) & 1;
-          if (!mbar_wait_bounded(p_full, (n - 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          mma_ts_tile(tmem_base + T_DQ, tmem_base + T_S, smem_u32(sStage + sp * 2 * TILE), n > 1);
-          mma_commit(&st_empty[sp]);
-        }
-        if (n < nk) {
-          const int st = n & 1;
-          if (!mbar_wait_bounded(&st_full[st], (n >> 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t sk = smem_u32(sStage + st * 2 * TILE);
-          mma_ss_tile(tmem_base + T_S, qA, sk);           // S = Q K^T
-          mma_ss_tile(tmem_base + T_DP, gA, sk + TILE);   // dP = dO V^T
-          mma_commit(s_full);
-        }
+      bool ok = mbar_wait_bounded(res_full, 0, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
+      if (ok) {
+        ok = mma_schedule(
+            N, st_full, st_empty, s_full, p_full, a,
+            [&](int n) {  // S = Q K_n^T, dP = dO V_n^T into buffer n & 1
+              const uint32_t st = smem_u32(sStage + (n % NST) * STAGE_Q);
+              const uint32_t buf = tmem_base + static_cast<uint32_t>((n & 1) * 128);
+              mma_ss_tile(buf, qA, st);
+              mma_ss_tile(buf + 64, gA, st + TILE_S);
+            },
+            [&](int n) {  // dQ += dS K_n
+              const uint32_t st = smem_u32(sStage + (n % NST) * STAGE_Q);
+              const uint32_t buf = tmem_base + static_cast<uint32_t>((n & 1) * 128);
+              mma_ts_tile(tmem_base + T_ACC0, buf, st, n > 0);
+            });
       }
       if (!ok) *abort_flag = 1;
       mma_commit(done_bar);
@@ -526,49 +543,48 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attn_bwd_dq_kernel(const __grid
     const float lse2 = a.lse[static_cast<int64_t>(bh) * a.S_pad + q];   // +inf past the sequence
     const float drow = a.Dv[static_cast<int64_t>(bh) * a.S_pad + q];
     bool ok = true;
-    for (int n = 0; n < nk && ok; ++n) {
+    for (int n = 0; n < N && ok; ++n) {
+      const int bsel = n & 1;
       if (!__all_sync(0xffffffffu,
-                      mbar_wait_bounded(s_full, n & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN))) {
+                      mbar_wait_bounded(&s_full[bsel], (n >> 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int k0 = n * BR;
+      const int k0 = n * BS;
       // keys k0 + j with j <= lim are seen by this row (causal, and inside the sequence)
-      const int lim = min(a.causal ? q - k0 : BR - 1, a.S - 1 - k0);
-      const bool whole = k0 + BR <= a.S && (!a.causal || k0 + BR - 1 <= q0);
+      const int lim = min(a.causal ? q - k0 : BS - 1, a.S - 1 - k0);
+      const bool whole = k0 + BS <= a.S && (!a.causal || k0 + BS - 1 <= q0);
+      const uint32_t buf = tmem_base + lane_off + static_cast<uint32_t>(bsel * 128);
+      uint32_t sv[2][32], gv[2][32];
+      tmem_ld_32x32b_x32(buf, sv[0]);
+      tmem_ld_32x32b_x32(buf + 32, sv[1]);
+      tmem_ld_32x32b_x32(buf + 64, gv[0]);
+      tmem_ld_32x32b_x32(buf + 96, gv[1]);
+      tmem_ld_wait();
+      uint32_t dk[32];
       float gmax = 0.f;
-#pragma unroll 1
-      for (int p = 0; p < 2; ++p) {
-        uint32_t sv[2][32], gv[2][32];
-        tmem_ld_32x32b_x32(tmem_base + lane_off + T_S + p * 64, sv[0]);
-        tmem_ld_32x32b_x32(tmem_base + lane_off + T_S + p * 64 + 32, sv[1]);
-        tmem_ld_32x32b_x32(tmem_base + lane_off + T_DP + p * 64, gv[0]);
-        tmem_ld_32x32b_x32(tmem_base + lane_off + T_DP + p * 64 + 32, gv[1]);
-        tmem_ld_wait();
-        uint32_t dk[32];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < 2; ++c) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float ds[2];
+        for (int i = 0; i < 16; ++i) {
+          float ds[2];
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int j = p * 64 + c * 32 + 2 * i + e;
-              float pv = ex2f(__uint_as_float(sv[c][2 * i + e]) * sl2 - lse2);
-              if (!whole && j > lim) pv = 0.f;
-              ds[e] = pv * (__uint_as_float(gv[c][2 * i + e]) - drow);
-              gmax = fmaxf(gmax, fabsf(ds[e]));
-            }
-            dk[c * 16 + i] = pack_f16x2(ds[0], ds[1]);
+          for (int e = 0; e < 2; ++e) {
+            const int j = c * 32 + 2 * i + e;
+            float pv = ex2f(__uint_as_float(sv[c][2 * i + e]) * sl2 - lse2);
+            if (!whole && j > lim) pv = 0.f;
+            ds[e] = pv * (__uint_as_float(gv[c][2 * i + e]) - drow);
+            gmax = fmaxf(gmax, fabsf(ds[e]));
           }
+          dk[c * 16 + i] = pack_f16x2(ds[0], ds[1]);
         }
-        tmem_st_32x32b_x32(tmem_base + lane_off + T_S + p * 32, dk);
       }
+      tmem_st_32x32b_x32(buf, dk);          // dS over the scores' first 32 columns
       note_f16_range(a.status, gmax, DEV_RANGE_ATTN_GRAD);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[bsel]);
     }
     if (!ok) {
       *abort_flag = 1;
@@ -576,7 +592,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attn_bwd_dq_kernel(const __grid
       tc_fence_after();
       uint32_t v[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tmem_base + lane_off + T_DQ + c * 32, v[c]);
+      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tmem_base + lane_off + T_ACC0 + c * 32, v[c]);
       tmem_ld_wait();
       if (q < a.S) {
         const int g = head / a.Hg, hl = head % a.Hg;
@@ -618,8 +634,8 @@ tp_status launch_attention_backward(const AttnBwdArgs& a, const uint16_t* dO, co
   const int nb = (a.S + BR - 1) / BR;
   if (a.S <= 0 || a.B == 0 || nh <= 0) return TP_OK;
   {
-    const int64_t warps = static_cast<int64_t>(a.B) * a.H * a.S_pad;
-    const unsigned blocks = static_cast<unsigned>((warps * 32 + 255) / 256);
+    const int64_t threads = static_cast<int64_t>(a.B) * a.H * a.S_pad * 16;
+    const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
     trace_before(stream, "attn_bwd_rowdot");
     const tp_status st = launch_ex(tp_attn_bwd_rowdot_kernel, dim3(blocks), dim3(256), 0, stream, 1, dO, O, o_f16,
                                    a.Dv, a.lse, a.B, a.S, a.H, a.S_pad);

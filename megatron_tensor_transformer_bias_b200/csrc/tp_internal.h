@@ -117,12 +117,15 @@ struct AttnArgs {
   uint64_t wait_limit_ns;
 };
 
-// Attention backward (tp_attention_bwd.cu).  Q, K, V [B*H][S][d] fp16 with boxes of 128
-// rows; dO [B*S, H*d] fp16 as a 4-D map (d, H, S, B), box {64, 1, 128, 1}; lse and Dv
-// [B*H][S_pad] fp32 (S_pad = S rounded up to 128); dqkv [B*S, ld_dqkv] bf16, head group
-// g's columns [g*3*Hg*d, ...) = [dQ heads | dK heads | dV heads].
+// Attention backward (tp_attention_bwd.cu).  Q, K, V [B*H][S][d] fp16; dO [B*S, H*d] fp16
+// as a 4-D map (d, H, S, B).  Maps of the resident 128-row tiles (box rows 128): tmQ, tmdO
+// (the dQ kernel), tmK, tmV (the dK/dV kernel); of the streamed 64-row sub-blocks (box rows
+// 64): tmQs, tmdOs (dK/dV), tmKs, tmVs (dQ).  lse and Dv [B*H][S_pad] fp32 (S_pad = S
+// rounded up to 128); dqkv [B*S, ld_dqkv] bf16, head group g's columns [g*3*Hg*d, ...) =
+// [dQ heads | dK heads | dV heads].
 struct AttnBwdArgs {
   CUtensorMap tmQ, tmK, tmV, tmdO;
+  CUtensorMap tmQs, tmKs, tmVs, tmdOs;
   float* lse;
   float* Dv;
   uint16_t* dqkv;
