@@ -286,7 +286,8 @@ TP_API tp_status tp_attn_forward(const void* X, int B, int S, int h, int heads, 
  * with fp32 accumulation; a P or dS value above 65504 sets TP_ERR_RANGE.  The
  * sums over rows, key blocks, query blocks and groups run in a fixed order:
  * results are bitwise reproducible on devices with the same SM count.  B*S == 0
- * zeroes dWqkv, dbqkv, dWo, dbo.  Limits: d == 128, heads % t == 0.
+ * zeroes dWqkv, dbqkv, dWo, dbo.  Limits: d == 128, heads % t == 0, S <= 65535*128
+ * (else TP_ERR_UNSUPPORTED).
  */
 TP_API size_t tp_attn_backward_workspace_bytes(int B, int S, int h, int heads, int d, int t);
 TP_API tp_status tp_attn_backward(const void* X, int B, int S, int h, int heads, int d, int t,

@@ -1022,6 +1022,7 @@ tp_status tp_attn_backward(const void* X, int B, int S, int h, int heads, int d,
   TP_TRY(check_shards(Wo, t, h, "Wo"));
   TP_TRY(check_bias_array(bqkv, t, "bqkv"));
   if (is_f16(Wqkv) || is_f16(Wo)) return fail(TP_ERR_UNSUPPORTED, "the backward pass takes bf16 Wqkv and Wo");
+  if (S > 65535 * 128) return fail(TP_ERR_UNSUPPORTED, "S > 65535 * 128 (the gradient kernels' grid)");
   if (M > 0 && (dX == X || dX == dY || dX == dX_add)) return fail(TP_ERR_INVALID_ARG, "dX aliases an input");
   const size_t need = tp_attn_backward_workspace_bytes(B, S, h, heads, d, t);
   if (need && (!ws || ws_bytes < need))

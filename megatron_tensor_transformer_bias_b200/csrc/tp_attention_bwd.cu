@@ -47,7 +47,8 @@ constexpr int TILE_R = 2 * HALF_R;           // 32 KB
 constexpr int HALF_S = BS * 64 * 2;          // [64 rows x 64 d]: 8 KB
 constexpr int TILE_S = 2 * HALF_S;           // 16 KB
 constexpr int NST = 4;                       // shared-memory stages of streamed sub-blocks
-constexpr int THREADS = 192;                 // warp 0 TMA, warp 1 MMA, warps 2..5 compute
+constexpr int THREADS = 224;                 // warp 0 TMA, warps 1 and 2 MMA, warps 3..6 compute
+constexpr int ISSUERS = 2;                   // MMA-issuing threads (one MMA costs one thread ~100 cycles)
 constexpr int COMPUTE_THREADS = 128;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC_SS = idesc_f16_f32(BR, BS, 0, 0);   // resident x streamed^T, both K-major
@@ -146,32 +147,45 @@ __device__ __forceinline__ void store_row_bf16(uint16_t* dst, const uint32_t (&v
   }
 }
 
-// The MMA thread's schedule, shared by both kernels: S and dP of sub-blocks 0 and 1 into
-// the two score buffers, then per sub-block n: (wait for its P / dS) the gradient MMAs of
-// n, release its stage, and S and dP of n + 2 into the buffer n just freed.
+// One MMA-issuing thread's schedule, shared by both kernels.  Each kernel has two such
+// threads with disjoint products: a single thread issues an MMA every ~100 cycles whatever
+// its size, half the tensor pipe's rate on these 64-wide tiles.  `issue_ss(n)` is this
+// thread's score product of sub-block n (into buffer n & 1), `issue_ts(n)` its gradient
+// product (when `has_ts`), issued once the compute warps have written P and dS of n; the
+// score product of n + 2 follows into the buffer n frees.  Every product reads or writes
+// only this thread's own columns of a buffer, so tensor-pipe order within the thread is
+// the only order needed.  Stage n is released by each thread once its last reader of that
+// stage completes (st_empty counts both threads), and s_full counts both score products.
 template <typename SS, typename TS>
 __device__ __forceinline__ bool mma_schedule(int N, uint64_t* st_full, uint64_t* st_empty, uint64_t* s_full,
-                                             uint64_t* p_full, const AttnBwdArgs& a, SS issue_ss, TS issue_ts) {
+                                             uint64_t* p_full, const AttnBwdArgs& a, bool has_ts, SS issue_ss,
+                                             TS issue_ts) {
   for (int n = 0; n < N && n < 2; ++n) {
     if (!mbar_wait_bounded(&st_full[n % NST], (n / NST) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN))
       return false;
     tc_fence_after();
     issue_ss(n);
     mma_commit(&s_full[n & 1]);
+    if (!has_ts) mma_commit(&st_empty[n % NST]);
   }
   for (int n = 0; n < N; ++n) {
     const int b = n & 1;
-    if (!mbar_wait_bounded(&p_full[b], (n >> 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN)) return false;
-    tc_fence_after();
-    issue_ts(n);
-    mma_commit(&st_empty[n % NST]);
     const int m = n + 2;
+    if (has_ts || m < N) {
+      if (!mbar_wait_bounded(&p_full[b], (n >> 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN)) return false;
+      tc_fence_after();
+    }
+    if (has_ts) {
+      issue_ts(n);
+      mma_commit(&st_empty[n % NST]);
+    }
     if (m < N) {
       if (!mbar_wait_bounded(&st_full[m % NST], (m / NST) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN))
         return false;
       tc_fence_after();
       issue_ss(m);
       mma_commit(&s_full[b]);
+      if (!has_ts) mma_commit(&st_empty[m % NST]);
     }
   }
   return true;
@@ -246,9 +260,12 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attn_bwd_dkdv_kernel(const __gr
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int kb = static_cast<int>(blockIdx.x);        // key block (causal: most query sub-blocks first)
-  const int head = a.head0 + static_cast<int>(blockIdx.y);
-  const int b = blockIdx.z;
+  // Key block in the slowest grid dimension: CTAs are dispatched in block order, so under the
+  // causal mask the longest ones (key block 0 sees every query) start first and the short
+  // ones fill the tail.
+  const int kb = static_cast<int>(blockIdx.z);
+  const int head = a.head0 + static_cast<int>(blockIdx.x);
+  const int b = blockIdx.y;
   const int bh = b * a.H + head;
   const int k0 = kb * BR;
   const int nsb_all = (a.S + BS - 1) / BS;
@@ -259,13 +276,13 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attn_bwd_dkdv_kernel(const __gr
     mbar_init(res_full, 1);
     for (int i = 0; i < NST; ++i) {
       mbar_init(&st_full[i], 1);
-      mbar_init(&st_empty[i], 1);
+      mbar_init(&st_empty[i], ISSUERS);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
+      mbar_init(&s_full[i], ISSUERS);
       mbar_init(&p_full[i], COMPUTE_THREADS);
     }
-    mbar_init(done_bar, 1);
+    mbar_init(done_bar, ISSUERS);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -315,24 +332,28 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attn_bwd_dkdv_kernel(const __gr
       for (int n = issued - NST > 0 ? issued - NST : 0; n < issued; ++n)
         mbar_wait_bounded(&st_full[n % NST], (n / NST) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
     }
-  } else if (warp == 1) {
+  } else if (warp <= ISSUERS) {
+    // issuer 0: S^T = K Q_n^T and dV += P^T dO_n (buffer columns 0..63);
+    // issuer 1: dP^T = V dO_n^T and dK += dS^T Q_n (buffer columns 64..127)
     if (lane == 0) {
-      const uint32_t kA = smem_u32(sK), vA = smem_u32(sV);
+      const uint32_t col = static_cast<uint32_t>((warp - 1) * 64);
+      const uint32_t resA = smem_u32(warp == 1 ? sK : sV);
+      const uint32_t ss_off = warp == 1 ? 0u : static_cast<uint32_t>(TILE_S);    // Q_n or dO_n
+      const uint32_t ts_off = warp == 1 ? static_cast<uint32_t>(TILE_S) : 0u;    // dO_n or Q_n
+      const uint32_t acc = tmem_base + (warp == 1 ? T_ACC0 : T_ACC1);
       bool ok = mbar_wait_bounded(res_full, 0, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
       if (ok) {
         ok = mma_schedule(
-            N, st_full, st_empty, s_full, p_full, a,
-            [&](int n) {  // S^T = K Q_n^T, dP^T = V dO_n^T into buffer n & 1
+            N, st_full, st_empty, s_full, p_full, a, true,
+            [&](int n) {
               const uint32_t st = smem_u32(sStage + (n % NST) * STAGE_KV);
-              const uint32_t buf = tmem_base + static_cast<uint32_t>((n & 1) * 128);
-              mma_ss_tile(buf, kA, st);
-              mma_ss_tile(buf + 64, vA, st + TILE_S);
+              const uint32_t buf = tmem_base + static_cast<uint32_t>((n & 1) * 128) + col;
+              mma_ss_tile(buf, resA, st + ss_off);
             },
-            [&](int n) {  // dV += P^T dO_n, dK += dS^T Q_n
+            [&](int n) {
               const uint32_t st = smem_u32(sStage + (n % NST) * STAGE_KV);
-              const uint32_t buf = tmem_base + static_cast<uint32_t>((n & 1) * 128);
-              mma_ts_tile(tmem_base + T_ACC0, buf, st + TILE_S, n > 0);
-              mma_ts_tile(tmem_base + T_ACC1, buf + 64, st, n > 0);
+              const uint32_t buf = tmem_base + static_cast<uint32_t>((n & 1) * 128) + col;
+              mma_ts_tile(acc, buf, st + ts_off, n > 0);
             });
       }
       if (!ok) *abort_flag = 1;
@@ -445,9 +466,9 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attn_bwd_dq_kernel(const __grid
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   const int nqb = (a.S + BR - 1) / BR;
-  const int qb = nqb - 1 - static_cast<int>(blockIdx.x);   // longest causal rows first
-  const int head = a.head0 + static_cast<int>(blockIdx.y);
-  const int b = blockIdx.z;
+  const int qb = nqb - 1 - static_cast<int>(blockIdx.z);   // longest causal rows dispatched first
+  const int head = a.head0 + static_cast<int>(blockIdx.x);
+  const int b = blockIdx.y;
   const int bh = b * a.H + head;
   const int q0 = qb * BR;
   const int nsb_all = (a.S + BS - 1) / BS;
@@ -457,13 +478,13 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attn_bwd_dq_kernel(const __grid
     mbar_init(res_full, 1);
     for (int i = 0; i < NST; ++i) {
       mbar_init(&st_full[i], 1);
-      mbar_init(&st_empty[i], 1);
+      mbar_init(&st_empty[i], ISSUERS);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
+      mbar_init(&s_full[i], ISSUERS);
       mbar_init(&p_full[i], COMPUTE_THREADS);
     }
-    mbar_init(done_bar, 1);
+    mbar_init(done_bar, ISSUERS);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -510,20 +531,22 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attn_bwd_dq_kernel(const __grid
       for (int n = issued - NST > 0 ? issued - NST : 0; n < issued; ++n)
         mbar_wait_bounded(&st_full[n % NST], (n / NST) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
     }
-  } else if (warp == 1) {
+  } else if (warp <= ISSUERS) {
+    // issuer 0: S = Q K_n^T and dQ += dS K_n (buffer columns 0..63); issuer 1: dP = dO V_n^T
     if (lane == 0) {
-      const uint32_t qA = smem_u32(sQ), gA = smem_u32(sdO);
+      const uint32_t col = static_cast<uint32_t>((warp - 1) * 64);
+      const uint32_t resA = smem_u32(warp == 1 ? sQ : sdO);
+      const uint32_t ss_off = warp == 1 ? 0u : static_cast<uint32_t>(TILE_S);    // K_n or V_n
       bool ok = mbar_wait_bounded(res_full, 0, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
       if (ok) {
         ok = mma_schedule(
-            N, st_full, st_empty, s_full, p_full, a,
-            [&](int n) {  // S = Q K_n^T, dP = dO V_n^T into buffer n & 1
+            N, st_full, st_empty, s_full, p_full, a, warp == 1,
+            [&](int n) {
               const uint32_t st = smem_u32(sStage + (n % NST) * STAGE_Q);
-              const uint32_t buf = tmem_base + static_cast<uint32_t>((n & 1) * 128);
-              mma_ss_tile(buf, qA, st);
-              mma_ss_tile(buf + 64, gA, st + TILE_S);
+              const uint32_t buf = tmem_base + static_cast<uint32_t>((n & 1) * 128) + col;
+              mma_ss_tile(buf, resA, st + ss_off);
             },
-            [&](int n) {  // dQ += dS K_n
+            [&](int n) {
               const uint32_t st = smem_u32(sStage + (n % NST) * STAGE_Q);
               const uint32_t buf = tmem_base + static_cast<uint32_t>((n & 1) * 128);
               mma_ts_tile(tmem_base + T_ACC0, buf, st, n > 0);
@@ -645,13 +668,13 @@ tp_status launch_attention_backward(const AttnBwdArgs& a, const uint16_t* dO, co
   {
     trace_before(stream, "attn_bwd_dkdv");
     const tp_status st =
-        launch_ex(tp_attn_bwd_dkdv_kernel, dim3(nb, nh, a.B), dim3(THREADS), DKDV_SMEM, stream, 1, a);
+        launch_ex(tp_attn_bwd_dkdv_kernel, dim3(nh, a.B, nb), dim3(THREADS), DKDV_SMEM, stream, 1, a);
     if (st != TP_OK) return st;
     trace_after(stream, "attn_bwd_dkdv");
   }
   {
     trace_before(stream, "attn_bwd_dq");
-    const tp_status st = launch_ex(tp_attn_bwd_dq_kernel, dim3(nb, nh, a.B), dim3(THREADS), DQ_SMEM, stream, 1, a);
+    const tp_status st = launch_ex(tp_attn_bwd_dq_kernel, dim3(nh, a.B, nb), dim3(THREADS), DQ_SMEM, stream, 1, a);
     if (st != TP_OK) return st;
     trace_after(stream, "attn_bwd_dq");
   }
