@@ -779,6 +779,9 @@ tp_status attn_backward_bf16(const void* X, int B, int S, int h, int H, int d, i
     TP_TRY(make_tmap_attn(&a.tmKs, w.fwd.k, B * H, S, d, 64));
     TP_TRY(make_tmap_attn(&a.tmVs, w.fwd.v, B * H, S, d, 64));
     TP_TRY(make_tmap_rows_by_head(&a.tmdOs, w.dO, B, S, H, d, 64));
+    TP_TRY(make_tmap_f16_3d(&a.tmOut, w.dqkv, static_cast<uint64_t>(3 * Hd), static_cast<uint64_t>(S),
+                            static_cast<uint64_t>(B), static_cast<uint64_t>(3 * Hd) * 2,
+                            static_cast<uint64_t>(S) * 3 * Hd * 2, 64, 128));
     a.lse = w.lse; a.Dv = w.Dv; a.dqkv = w.dqkv; a.ld_dqkv = 3 * Hd;
     a.B = B; a.S = S; a.H = H; a.Hg = Hg; a.head0 = 0; a.causal = causal; a.S_pad = static_cast<int>(S_pad);
     a.scale_log2 = scale_log2; a.scale = 1.f / sqrtf(static_cast<float>(d));

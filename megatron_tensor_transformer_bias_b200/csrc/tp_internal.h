@@ -126,6 +126,7 @@ struct AttnArgs {
 struct AttnBwdArgs {
   CUtensorMap tmQ, tmK, tmV, tmdO;
   CUtensorMap tmQs, tmKs, tmVs, tmdOs;
+  CUtensorMap tmOut;   // dqkv seen as (3*H*d, S, B) bf16, box {64, 128, 1}: the gradient blocks' TMA stores
   float* lse;
   float* Dv;
   uint16_t* dqkv;
