@@ -348,9 +348,9 @@ class FFNBwd(Workload):
         M, h, f, t = w.M, w.h, w.f, w.t
         self.kernel_amount = {k: ("tensor", 2 * M * h * f, "FLOP") for k in
                               ("gemm_bwd_recompute", "gemm_bwd_dz", "gemm_bwd_dw2", "gemm_bwd_dw1", "gemm_bwd_dx")}
-        # Each step traces four colsum launches: a chunk pass and a final pass for db1 (over dZ)
-        # and for db2 (over dY); their bytes, M*f*2 + M*h*2 in all, are spread over the four.
-        self.kernel_amount["colsum"] = ("hbm", (M * f * 2 + M * h * 2) // 4, "B")
+        # Each step traces two colsum launches, db1 (over dZ) and db2 (over dY); their bytes,
+        # M*f*2 + M*h*2 in all, are spread over the two.
+        self.kernel_amount["colsum"] = ("hbm", (M * f * 2 + M * h * 2) // 2, "B")
 
     def setup(self, dev, rank):
         import torch

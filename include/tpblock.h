@@ -195,7 +195,7 @@ TP_API tp_status tp_ffn_forward_noalloc(const void* X, int64_t M, int64_t h, int
  *           is 1 for z > 0, else 0).
  *  ws       tp_ffn_backward_workspace_bytes(...) bytes, 256-byte aligned:
  *           act(Z) (bf16), act'(Z) (fp16, in [-0.17, 1.13] for GeLU) and dZ
- *           (bf16), each [M, f], and the column sums' scratch.
+ *           (bf16), each [M, f].
  * The sums over rows (dW, db) and over shards (dX) are taken in a fixed
  * order: results are bitwise reproducible on devices with the same SM count.
  * M == 0 zeroes dW1, dW2, db1, db2.  Limits as tp_ffn_forward's bf16 path.
@@ -281,7 +281,7 @@ TP_API tp_status tp_attn_forward(const void* X, int B, int S, int h, int heads, 
  *  dbo      [h] fp32 out or NULL.
  *  ws       tp_attn_backward_workspace_bytes(...) bytes, 256-byte aligned: Q, K, V,
  *           O (fp16 / bf16), dO (fp16), dQKV (bf16), the rows' log-sum-exp and
- *           rowsum(dO * O) (fp32) and the column sums' scratch.
+ *           rowsum(dO * O) (fp32).
  * The attention gradients' tensor-core operands (P, dS, dO, Q, K, V) are fp16
  * with fp32 accumulation; a P or dS value above 65504 sets TP_ERR_RANGE.  The
  * sums over rows, key blocks, query blocks and groups run in a fixed order:

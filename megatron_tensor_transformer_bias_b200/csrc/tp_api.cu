@@ -472,22 +472,21 @@ tp_status validate_ffn(const void* X, int64_t M, int64_t h, int64_t f, int t, co
 }
 
 // ---------------------------------------------------------------- FFN backward (bf16)
-// Workspace: act(Z) [M, f] bf16 | act'(Z) [M, f] fp16 | dZ [M, f] bf16 | column-sum scratch.
+// Workspace: act(Z) [M, f] bf16 | act'(Z) [M, f] fp16 | dZ [M, f] bf16.
 struct FfnBwdWs {
   uint16_t *A, *G, *dZ;
-  float* part;
 };
 
 size_t ffn_bwd_ws_bytes(int64_t M, int64_t h, int64_t f) {
+  (void)h;
   const size_t mf = align_up(static_cast<size_t>(M) * f * 2);
-  return 3 * mf + align_up(colsum_workspace_bytes(M, f > h ? f : h));
+  return 3 * mf;
 }
 
 FfnBwdWs ffn_bwd_ws_layout(void* ws, int64_t M, int64_t f) {
   const size_t mf = align_up(static_cast<size_t>(M) * f * 2);
   uint8_t* p = static_cast<uint8_t*>(ws);
-  return {reinterpret_cast<uint16_t*>(p), reinterpret_cast<uint16_t*>(p + mf), reinterpret_cast<uint16_t*>(p + 2 * mf),
-          reinterpret_cast<float*>(p + 3 * mf)};
+  return {reinterpret_cast<uint16_t*>(p), reinterpret_cast<uint16_t*>(p + mf), reinterpret_cast<uint16_t*>(p + 2 * mf)};
 }
 
 tp_status ffn_backward_bf16(const void* X, int64_t M, int64_t h, int64_t f, int t, const tp_shard* W1,
@@ -572,8 +571,8 @@ tp_status ffn_backward_bf16(const void* X, int64_t M, int64_t h, int64_t f, int 
     TP_TRY(launch_gemm(a, stream, "gemm_bwd_dx"));
   }
   // 6. bias gradients: column sums of dZ and dY in a fixed order
-  if (db1) TP_TRY(launch_colsum(w.dZ, M, f, f, w.part, db1, stream));
-  if (db2) TP_TRY(launch_colsum(dY, M, h, h, w.part, db2, stream));
+  if (db1) TP_TRY(launch_colsum(w.dZ, M, f, f, db1, stream));
+  if (db2) TP_TRY(launch_colsum(dY, M, h, h, db2, stream));
   return TP_OK;
 }
 
@@ -664,7 +663,6 @@ struct AttnBwdWs {
   uint16_t* dqkv;      // [M, 3*H*d] bf16, head groups' [dQ | dK | dV] column blocks
   float* lse;          // [B*H][S_pad]
   float* Dv;           // [B*H][S_pad]
-  float* colsum;       // column-sum scratch
 };
 
 int64_t attn_s_pad(int64_t S) { return (S + 127) / 128 * 128; }
@@ -672,8 +670,8 @@ int64_t attn_s_pad(int64_t S) { return (S + 127) / 128 * 128; }
 size_t attn_bwd_ws_bytes(int64_t B, int64_t S, int64_t h, int64_t H, int64_t d) {
   const size_t qkv = align_up(static_cast<size_t>(B) * S * H * d * 2);
   const size_t vec = align_up(static_cast<size_t>(B) * H * attn_s_pad(S) * 4);
-  const int64_t cs = 3 * H * d > h ? 3 * H * d : h;
-  return 4 * qkv + qkv + 3 * qkv + 2 * vec + align_up(colsum_workspace_bytes(B * S, cs));
+  (void)h;
+  return 4 * qkv + qkv + 3 * qkv + 2 * vec;
 }
 
 AttnBwdWs attn_bwd_ws_layout(void* ws, int64_t B, int64_t S, int64_t H, int64_t d) {
@@ -686,7 +684,6 @@ AttnBwdWs attn_bwd_ws_layout(void* ws, int64_t B, int64_t S, int64_t H, int64_t 
   w.dqkv = reinterpret_cast<uint16_t*>(p + 5 * qkv);
   w.lse = reinterpret_cast<float*>(p + 8 * qkv);
   w.Dv = reinterpret_cast<float*>(p + 8 * qkv + vec);
-  w.colsum = reinterpret_cast<float*>(p + 8 * qkv + 2 * vec);
   return w;
 }
 
@@ -737,7 +734,7 @@ tp_status attn_backward_bf16(const void* X, int B, int S, int h, int H, int d, i
     TP_TRY(launch_attention(a, stream));
   }
   // 3. dbo = column sums of dY
-  if (dbo) TP_TRY(launch_colsum(dY, M, h, h, w.colsum, dbo, stream));
+  if (dbo) TP_TRY(launch_colsum(dY, M, h, h, dbo, stream));
   // 4. dWo_i = O_i^T dY (rows i*n.. of dWo): the row-parallel projection's weight gradient
   {
     GemmArgs a;
@@ -804,7 +801,7 @@ tp_status attn_backward_bf16(const void* X, int B, int S, int h, int H, int d, i
     TP_TRY(launch_gemm(a, stream, "gemm_attn_bwd_dwqkv"));
   }
   // 8. dbqkv = column sums of dQKV
-  if (dbqkv) TP_TRY(launch_colsum(w.dqkv, M, 3 * Hd, 3 * Hd, w.colsum, dbqkv, stream));
+  if (dbqkv) TP_TRY(launch_colsum(w.dqkv, M, 3 * Hd, 3 * Hd, dbqkv, stream));
   // 9. dX = sum_i dQKV_i Wqkv_i^T (+ dX_add): the sum over head groups, in one accumulator
   {
     GemmArgs a;

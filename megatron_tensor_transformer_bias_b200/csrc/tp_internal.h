@@ -174,11 +174,8 @@ tp_status launch_ffn_fp32(const float* X, int64_t M, int64_t h, int64_t f, int t
                           const void* const* b1, const tp_shard* W2, const float* b2, const float* resid,
                           float* out, int act, float* Z, float* P, cudaStream_t stream);
 tp_status launch_selftest_wait(uint64_t limit_ns, cudaStream_t stream);
-// out[c] = sum_r x[r, c] (bf16 x [M, ld], fp32 out [n]) in a fixed order, through `part`
-// (colsum_workspace_bytes(M, n) bytes of fp32 scratch).
-size_t colsum_workspace_bytes(int64_t M, int64_t n);
-tp_status launch_colsum(const void* x, int64_t M, int64_t n, int64_t ld, float* part, float* out,
-                        cudaStream_t stream);
+// out[c] = sum_r x[r, c] (bf16 x [M, ld], fp32 out [n]) in a fixed order, one pass, no scratch.
+tp_status launch_colsum(const void* x, int64_t M, int64_t n, int64_t ld, float* out, cudaStream_t stream);
 tp_status launch_act(const float* x, float* y, int64_t n, int act, cudaStream_t stream);
 
 // Record `msg` as the calling thread's tp_last_error() and return `s`.

@@ -218,19 +218,31 @@ __global__ void __launch_bounds__(256) act_kernel(const float* __restrict__ x, f
 // in turn, then the 8 warps' sums are added in the order 0..7); pass 2 adds the chunks'
 // sums in the order 0, 1, ...  Each thread of pass 1 owns 8 adjacent columns (one
 // 16-byte load per row), so a warp reads 512 contiguous bytes of a row.
-constexpr int CS_ROWS = 128;
-constexpr int CS_COLS = 256;   // 32 lanes x 8 columns
-
-__global__ void __launch_bounds__(256) colsum_chunk_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t n,
-                                                           int64_t ld, float* __restrict__ part) {
-  __shared__ float red[8][CS_COLS];
-  const int w = threadIdx.x / 32, l = threadIdx.x % 32;
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * CS_COLS + l * 8;
-  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * CS_ROWS;
+// Column sums of a bf16 [M, n] matrix (row stride ld) in one launch: a cluster of 8 CTAs owns
+// 128 columns, CTA q of it the rows [q R, (q + 1) R) with R = ceil(M / 8); in a CTA, row slot
+// k = 2 w + (lane / 16) of warp w reads rows k, k + 16, ... of its range (256 contiguous
+// bytes per row, 8 columns per lane) and sums them in increasing order; the 16 slots' sums
+// add up in order 0..15, and CTA 0 of the cluster adds the 8 CTAs' sums in order 0..7 through
+// distributed shared memory.  Fixed order throughout: the result does not depend on timing.
+constexpr int CS_COLS = 128;    // 16 lanes x 8 columns
+constexpr int CS_SLOTS = 16;    // rows read at once by a CTA: 8 warps x 2
+constexpr int CS_SPLIT = 8;     // CTAs (row ranges) per cluster
+__global__ void __launch_bounds__(256) colsum_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t n,
+                                                     int64_t ld, float* __restrict__ out) {
+  __shared__ float red[CS_SLOTS][CS_COLS];
+  __shared__ float psum[CS_COLS];
+  const int slot = threadIdx.x / 16, l16 = threadIdx.x % 16;
+  const uint32_t q = cluster_ctarank();
+  const int64_t cb = blockIdx.x / CS_SPLIT;
+  const int64_t c0 = cb * CS_COLS + l16 * 8;
+  const int64_t rows = (M + CS_SPLIT - 1) / CS_SPLIT;
+  const int64_t r_lo = static_cast<int64_t>(q) * rows;
+  const int64_t r_hi = r_lo + rows < M ? r_lo + rows : M;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   pdl_wait();
   if (c0 < n) {
-    for (int64_t r = r0 + w; r < r0 + CS_ROWS && r < M; r += 8) {
+#pragma unroll 4
+    for (int64_t r = r_lo + slot; r < r_hi; r += CS_SLOTS) {
       float f[8];
       load_bf16x8(x + r * ld + c0, f);
 #pragma unroll
@@ -238,27 +250,30 @@ __global__ void __launch_bounds__(256) colsum_chunk_kernel(const uint16_t* __res
     }
   }
 #pragma unroll
-  for (int j = 0; j < 8; ++j) red[w][l * 8 + j] = acc[j];
+  for (int j = 0; j < 8; ++j) red[slot][l16 * 8 + j] = acc[j];
   __syncthreads();
-  const int64_t c = static_cast<int64_t>(blockIdx.x) * CS_COLS + threadIdx.x;
-  if (c < n) {
+  if (threadIdx.x < CS_COLS) {
     float v = red[0][threadIdx.x];
 #pragma unroll
-    for (int i = 1; i < 8; ++i) v += red[i][threadIdx.x];
-    part[static_cast<int64_t>(blockIdx.y) * n + c] = v;
+    for (int i = 1; i < CS_SLOTS; ++i) v += red[i][threadIdx.x];
+    psum[threadIdx.x] = v;
   }
-  pdl_launch_dependents();
-}
-
-__global__ void __launch_bounds__(256) colsum_final_kernel(const float* __restrict__ part, int chunks, int64_t n,
-                                                           float* __restrict__ out) {
-  pdl_wait();
-  const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (c < n) {
-    float v = part[c];
-    for (int i = 1; i < chunks; ++i) v += part[static_cast<int64_t>(i) * n + c];
-    out[c] = v;
+  cluster_sync_all();   // every CTA's psum is written and visible to the cluster
+  if (q == 0 && threadIdx.x < CS_COLS) {
+    const int64_t c = cb * CS_COLS + threadIdx.x;
+    if (c < n) {
+      float v = psum[threadIdx.x];
+      const uint32_t own = smem_u32(&psum[threadIdx.x]);
+#pragma unroll
+      for (uint32_t k = 1; k < CS_SPLIT; ++k) {
+        float pk;
+        asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(pk) : "r"(mapa_shared(own, k)) : "memory");
+        v += pk;
+      }
+      out[c] = v;
+    }
   }
+  cluster_sync_all();   // the other CTAs' shared memory stays until CTA 0 has read it
   pdl_launch_dependents();
 }
 
@@ -498,25 +513,15 @@ tp_status launch_act(const float* x, float* y, int64_t n, int act, cudaStream_t 
   return TP_OK;
 }
 
-size_t colsum_workspace_bytes(int64_t M, int64_t n) {
-  return static_cast<size_t>((M + CS_ROWS - 1) / CS_ROWS) * static_cast<size_t>(n) * sizeof(float);
-}
-
-tp_status launch_colsum(const void* x, int64_t M, int64_t n, int64_t ld, float* part, float* out,
-                        cudaStream_t stream) {
+tp_status launch_colsum(const void* x, int64_t M, int64_t n, int64_t ld, float* out, cudaStream_t stream) {
   if (n == 0) return TP_OK;
-  const int chunks = static_cast<int>((M + CS_ROWS - 1) / CS_ROWS);
-  if (chunks == 0) {
+  if (M == 0) {
     const cudaError_t e = cudaMemsetAsync(out, 0, static_cast<size_t>(n) * sizeof(float), stream);
     return e == cudaSuccess ? TP_OK : set_error(TP_ERR_CUDA, cudaGetErrorString(e));
   }
   trace_before(stream, "colsum");
-  TP_TRY_LAUNCH(launch_ex(colsum_chunk_kernel, dim3(static_cast<unsigned>((n + CS_COLS - 1) / CS_COLS), chunks),
-                          dim3(256), 0, stream, 1, static_cast<const uint16_t*>(x), M, n, ld, part));
-  trace_after(stream, "colsum");
-  trace_before(stream, "colsum");
-  TP_TRY_LAUNCH(launch_ex(colsum_final_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, stream, 1,
-                          static_cast<const float*>(part), chunks, n, out));
+  TP_TRY_LAUNCH(launch_ex(colsum_kernel, dim3(static_cast<unsigned>((n + CS_COLS - 1) / CS_COLS * CS_SPLIT)),
+                          dim3(256), 0, stream, CS_SPLIT, static_cast<const uint16_t*>(x), M, n, ld, out));
   trace_after(stream, "colsum");
   return TP_OK;
 }

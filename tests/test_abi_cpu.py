@@ -53,7 +53,7 @@ def test_workspace_sizes(L):
     assert L.tp_row_linear_workspace_bytes(M, h, t, tb.TP_REDUCE_FUSED) == 0
     assert L.tp_row_linear_workspace_bytes(M, h, t, tb.TP_REDUCE_PARTIALS) == t * M * h * 4 + ctr
     mf = M * f * 2
-    assert tb.tp_ffn_backward_workspace_bytes(M, h, f, t) == 3 * mf + (M + 127) // 128 * f * 4
+    assert tb.tp_ffn_backward_workspace_bytes(M, h, f, t) == 3 * mf   # act(Z), act'(Z), dZ
     assert tb.tp_ffn_backward_workspace_bytes(0, h, f, t) == 0
     B, S, H, d = 2, 2048, 32, 128
     q = B * S * H * d * 2
@@ -198,8 +198,7 @@ def test_attn_backward_workspace_and_validation(L):
     B, S, h, H, d, t = 2, 2048, 4096, 32, 128, 4
     q = B * S * H * d * 2
     vec = B * H * 2048 * 4
-    colsum = (B * S + 127) // 128 * (3 * H * d) * 4
-    assert tb.tp_attn_backward_workspace_bytes(B, S, h, H, d, t) == 8 * q + 2 * vec + colsum
+    assert tb.tp_attn_backward_workspace_bytes(B, S, h, H, d, t) == 8 * q + 2 * vec
     assert tb.tp_attn_backward_workspace_bytes(0, S, h, H, d, t) == 0
     # S not a multiple of 128: the row vectors are padded to whole 128-query blocks
     assert tb.tp_attn_backward_workspace_bytes(1, 200, 256, 2, d, 1) >= 8 * (200 * 2 * d * 2) + 2 * 2 * 256 * 4
