@@ -724,29 +724,48 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
 // full barrier; the leader's commits arrive on both CTAs' empty / accumulator
 // barriers; both CTAs' epilogues arrive on the leader's accumulator-empty barrier.
 // No load is multicast.
+//
+// A wide variant (PBN = 512: 256 x 512 tiles) serves grids whose 256 x 256 tiles would
+// take more than one round but whose 256 x 512 tiles fit in one: each 64-wide K step
+// feeds two N=256 MMAs from one A tile, so an SM streams 48 KB per 1024 tensor cycles
+// instead of 32 KB per 512 (a quarter fewer operand bytes for the same work).  Its one
+// accumulator fills all 512 TMEM columns (no epilogue/main-loop overlap across tiles,
+// which a one-round grid does not have).
 constexpr int P_ROWS = 2 * BM;                      // 256 rows per pair
-constexpr int P_STAGES = 6;
 constexpr int P_A_BYTES = BM * BK * 2;              // 16 KB per CTA
-constexpr int P_B_BYTES = (BN / 2) * BK * 2;        // 16 KB per CTA
-constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
-constexpr int P_SMEM_BYTES = 1024 + P_STAGES * P_STAGE_BYTES + STAGING_BYTES + 256;
 
-template <int EPI, int OPL>
+template <int PBN>
+struct PairCfg {
+  static_assert(PBN == 256 || PBN == 512, "pair tile width");
+  static constexpr int NH = PBN / 256;                      // N=256 MMAs per 16-deep K step
+  static constexpr int B_BYTES = (PBN / 2) * BK * 2;        // this CTA's B columns: 16 or 32 KB
+  static constexpr int STAGE_BYTES = P_A_BYTES + B_BYTES;
+  static constexpr int STAGES = PBN == 256 ? 6 : 4;
+  static constexpr int NUM_ACC = TMEM_COLS / PBN;           // 2 or 1
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + 256;
+};
+static_assert(PairCfg<256>::SMEM_BYTES == PairCfg<512>::SMEM_BYTES, "both widths share the smem attribute");
+constexpr int P_SMEM_BYTES = PairCfg<256>::SMEM_BYTES;
+
+template <int EPI, int OPL, int PBN>
 __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_constant__ GemmArgs a) {
+  using C = PairCfg<PBN>;
   constexpr bool A_MN = (OPL & OPL_A_MN) != 0;
   constexpr bool B_KM = (OPL & OPL_B_KMAJOR) != 0;
+  // the in-epilogue partials reduction counts 128-column regions of 256-wide tiles
+  static_assert(PBN == 256 || EPI != EPI_PARTIAL_F32, "wide tiles: no partials epilogue");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sA = smem;
-  uint8_t* sB = smem + P_STAGES * P_A_BYTES;
-  uint8_t* staging = smem + P_STAGES * P_STAGE_BYTES;
+  uint8_t* sB = smem + C::STAGES * P_A_BYTES;
+  uint8_t* staging = smem + C::STAGES * C::STAGE_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(staging + STAGING_BYTES);
-  uint64_t* full_bar = bars;                             // [P_STAGES], used in the leader
-  uint64_t* empty_bar = bars + P_STAGES;                 // [P_STAGES], both CTAs
-  uint64_t* acc_full = bars + 2 * P_STAGES;              // [NUM_ACC], both CTAs
-  uint64_t* acc_empty = bars + 2 * P_STAGES + NUM_ACC;   // [NUM_ACC], used in the leader
-  uint64_t* drain_bar = bars + 2 * P_STAGES + 2 * NUM_ACC;
+  uint64_t* full_bar = bars;                                    // [STAGES], used in the leader
+  uint64_t* empty_bar = bars + C::STAGES;                       // [STAGES], both CTAs
+  uint64_t* acc_full = bars + 2 * C::STAGES;                    // [NUM_ACC], both CTAs
+  uint64_t* acc_empty = bars + 2 * C::STAGES + C::NUM_ACC;      // [NUM_ACC], used in the leader
+  uint64_t* drain_bar = bars + 2 * C::STAGES + 2 * C::NUM_ACC;
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
 
@@ -758,17 +777,17 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
   const int nclusters = static_cast<int>(gridDim.x >> 1);
 
   const int m_tiles = (a.M + P_ROWS - 1) / P_ROWS;
-  const int n_tiles = (a.N + BN - 1) / BN;
+  const int n_tiles = (a.N + PBN - 1) / PBN;
   const int num_tiles = m_tiles * n_tiles * (a.concat ? 1 : a.G);
   const int kb_per_group = (a.Kg + BK - 1) / BK;   // a ragged last K step reads zero fill
   const int k_iters = a.concat ? kb_per_group * a.G : kb_per_group;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < P_STAGES; ++s) {
+    for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
-    for (int s = 0; s < NUM_ACC; ++s) {
+    for (int s = 0; s < C::NUM_ACC; ++s) {
       mbar_init(&acc_full[s], 1);
       mbar_init(&acc_empty[s], 2 * EPI_WARPS);  // one arrival per epilogue warp of each CTA
     }
@@ -804,9 +823,9 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
       if (cid < num_tiles) {
         const TileCoord tc = tile_coord(a, cid, m_tiles, n_tiles);
         const int m0 = tc.m_blk * P_ROWS + static_cast<int>(rank) * BM;
-        const int n0 = tc.n_blk * BN + static_cast<int>(rank) * (BN / 2);
+        const int n0 = tc.n_blk * PBN + static_cast<int>(rank) * 128;
         const bool rev = a.concat != 0;
-        const int pre = k_iters < P_STAGES ? k_iters : P_STAGES;
+        const int pre = k_iters < C::STAGES ? k_iters : C::STAGES;
         for (int it = 0; it < pre; ++it) {
           const int kidx = rev ? k_iters - 1 - it : it;
           const int g = a.concat ? kidx / kb_per_group : tc.g;
@@ -814,8 +833,11 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
           const int ka = g * a.a_k_per_group + kb * BK;
           if (!A_MN) tma_prefetch_l2_2d(&a.tmA, ka, m0);
           else tma_prefetch_l2_3d(&a.tmA, 0, ka, (g * a.a_m_per_group + m0) / 64);
-          if (!B_KM) tma_prefetch_l2_3d(&a.tmB[g], 0, kb * BK, n0 / 64);
-          else tma_prefetch_l2_2d(&a.tmB[g], kb * BK, n0);
+#pragma unroll
+          for (int h = 0; h < C::NH; ++h) {
+            if (!B_KM) tma_prefetch_l2_3d(&a.tmB[g], 0, kb * BK, (n0 + h * 256) / 64);
+            else tma_prefetch_l2_2d(&a.tmB[g], kb * BK, n0 + h * 256);
+          }
         }
       }
       pdl_wait();  // the previous kernel's outputs (our operands) are complete
@@ -826,7 +848,8 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
       for (int tile = cid; tile < num_tiles && ok; tile += nclusters) {
         const TileCoord tc = tile_coord(a, tile, m_tiles, n_tiles);
         const int m0 = tc.m_blk * P_ROWS + static_cast<int>(rank) * BM;
-        const int n0 = tc.n_blk * BN + static_cast<int>(rank) * (BN / 2);
+        // this CTA's B columns: [n0 + h*256, +128) for each N=256 half h of the tile
+        const int n0 = tc.n_blk * PBN + static_cast<int>(rank) * 128;
         // Row layer: the K loop runs backwards in even rounds of tiles and forwards in odd
         // ones, so each round starts on the K-slices of A that are still in L2 -- the end
         // of K for the first round (the producing layer wrote it last), the start for the
@@ -841,7 +864,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
           const int g = a.concat ? kidx / kb_per_group : tc.g;
           const int kb = a.concat ? kidx - g * kb_per_group : kidx;
           const uint32_t fb = full0_leader + static_cast<uint32_t>(stage) * 8u;
-          if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * P_STAGE_BYTES);
+          if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * C::STAGE_BYTES);
           uint8_t* a_dst = sA + stage * P_A_BYTES;
           const int ka = g * a.a_k_per_group + kb * BK;
           if (!A_MN) {
@@ -849,31 +872,34 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
           } else {  // two 64-wide M blocks of 64 K rows, one load
             tma_load_3d_pair(a_dst, &a.tmA, fb, 0, ka, (g * a.a_m_per_group + m0) / 64, pol_a);
           }
-          uint8_t* b_dst = sB + stage * P_B_BYTES;
-          if (!B_KM) {  // this CTA's two 64-wide N blocks of 64 K rows, one load
-            tma_load_3d_pair(b_dst, &a.tmB[g], fb, 0, kb * BK, n0 / 64, pol_b);
-          } else {  // this CTA's 128 N rows, 64 K each
-            tma_load_2d_pair(b_dst, &a.tmB[g], fb, kb * BK, n0, pol_b);
+          uint8_t* b_dst = sB + stage * C::B_BYTES;
+#pragma unroll
+          for (int h = 0; h < C::NH; ++h) {
+            if (!B_KM) {  // this CTA's two 64-wide N blocks of 64 K rows, one load
+              tma_load_3d_pair(b_dst + h * 16384, &a.tmB[g], fb, 0, kb * BK, (n0 + h * 256) / 64, pol_b);
+            } else {  // this CTA's 128 N rows, 64 K each
+              tma_load_2d_pair(b_dst + h * 16384, &a.tmB[g], fb, kb * BK, n0 + h * 256, pol_b);
+            }
           }
           ++issued;
-          if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
       }
       // Our copies are in flight until the leader's MMAs have consumed their stage:
-      // wait for the consumption of the last min(issued, P_STAGES) stages.
-      const int pending = issued < P_STAGES ? issued : P_STAGES;
+      // wait for the consumption of the last min(issued, STAGES) stages.
+      const int pending = issued < C::STAGES ? issued : C::STAGES;
       int s = stage;
       uint32_t ph = phase;
       for (int i = 0; i < pending; ++i) {
-        if (--s < 0) { s = P_STAGES - 1; ph ^= 1u; }
+        if (--s < 0) { s = C::STAGES - 1; ph ^= 1u; }
         mbar_wait_bounded(&empty_bar[s], ph, a.wait_limit_ns, a.status, WAIT_SITE_PRODUCER);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader only)
     if (lane == 0 && leader) {
-      const uint32_t idesc = a.ab_f16 ? idesc_f16_f32(P_ROWS, BN, A_MN, !B_KM)
-                                      : idesc_bf16_f32(P_ROWS, BN, A_MN, !B_KM);
+      const uint32_t idesc = a.ab_f16 ? idesc_f16_f32(P_ROWS, 256, A_MN, !B_KM)
+                                      : idesc_bf16_f32(P_ROWS, 256, A_MN, !B_KM);
       const uint32_t sA_addr = smem_u32(sA);
       const uint32_t sB_addr = smem_u32(sB);
       int stage = 0;
@@ -886,7 +912,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
           *abort_flag = 1; ok = false; break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * PBN);
         for (int it = 0; it < k_iters; ++it) {
           if (*abort_flag) { ok = false; break; }
           if (!mbar_wait_bounded(&full_bar[stage], phase, a.wait_limit_ns, a.status, WAIT_SITE_MMA_FULL)) {
@@ -894,21 +920,25 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
           }
           tc_fence_after();
           const uint32_t a_base = sA_addr + stage * P_A_BYTES;
-          const uint32_t b_base = sB_addr + stage * P_B_BYTES;
+          const uint32_t b_base = sB_addr + stage * C::B_BYTES;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t adesc = A_MN ? smem_desc_sw128(a_base + k * 16 * 128, B_BLOCK_BYTES, 1024)
                                           : smem_desc_sw128(a_base + k * 32, 16, 1024);
-            const uint64_t bdesc = B_KM ? smem_desc_sw128(b_base + k * 32, 16, 1024)
-                                              : smem_desc_sw128(b_base + k * 16 * 128, B_BLOCK_BYTES, 1024);
-            mma_pair_ss(d_tmem, adesc, bdesc, idesc, (it > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+            for (int h = 0; h < C::NH; ++h) {
+              const uint32_t bh = b_base + static_cast<uint32_t>(h) * 16384u;
+              const uint64_t bdesc = B_KM ? smem_desc_sw128(bh + k * 32, 16, 1024)
+                                          : smem_desc_sw128(bh + k * 16 * 128, B_BLOCK_BYTES, 1024);
+              mma_pair_ss(d_tmem + static_cast<uint32_t>(h * 256), adesc, bdesc, idesc, (it > 0 || k > 0) ? 1u : 0u);
+            }
           }
           mma_commit_pair_mask(&empty_bar[stage], 0x3);  // frees this stage in both CTAs
-          if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
         mma_commit_pair_mask(&acc_full[acc], 0x3);       // accumulator ready in both CTAs
-        if (++acc == NUM_ACC) { acc = 0; acc_phase ^= 1u; }
+        if (++acc == C::NUM_ACC) { acc = 0; acc_phase ^= 1u; }
       }
       mma_commit_pair_local(drain_bar);
       mbar_wait_bounded(drain_bar, 0, a.wait_limit_ns, a.status, WAIT_SITE_MMA_ACC);
@@ -917,7 +947,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
     // ------------------------------------------------------------ epilogue (warps 2..5 of both CTAs)
     const int sub = warp & 3;
     const int row_in_tile = static_cast<int>(rank) * BM + sub * 32 + lane;
-    const int col_half = (warp - 2) / 4;    // columns [col_half*BN/2, +BN/2) of each tile
+    const int col_half = (warp - 2) / 4;    // columns [col_half*PBN/2, +PBN/2) of each tile
     const uint32_t acc_empty0_leader = mapa_shared(smem_u32(&acc_empty[0]), 0);
     pdl_wait();  // bias / residual inputs and our outputs: after the previous kernel completes
     int acc = 0;
@@ -938,12 +968,12 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
       tc_fence_after();
       const TileCoord tc = tile_coord(a, tile, m_tiles, n_tiles);
       const int row = tc.m_blk * P_ROWS + row_in_tile;
-      const int n0 = tc.n_blk * BN;
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const int n0 = tc.n_blk * PBN;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(acc * PBN);
       // columns [c_begin*32, c_end*32) of the tile, clipped to N (a multiple of 32);
       // the TMEM load of chunk c+1 is issued before chunk c is processed
-      const int c_begin = col_half * (BN / 64);
-      int c_end = (col_half + 1) * (BN / 64);
+      const int c_begin = col_half * (PBN / 64);
+      int c_end = (col_half + 1) * (PBN / 64);
       if (n0 + c_end * 32 > a.N) c_end = (a.N - n0) / 32;
       // partials mode with the reduction here: this warp's region and its role in it
       const int row0 = tc.m_blk * P_ROWS + static_cast<int>(rank) * BM + sub * 32;
@@ -970,7 +1000,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
         uint32_t r[2][32];
         tmem_ld_32x32b_x32(t_row + c_begin * 32, r[0]);
 #pragma unroll
-        for (int c = c_begin; c < c_begin + BN / 64; ++c) {
+        for (int c = c_begin; c < c_begin + PBN / 64; ++c) {
           if (c >= c_end) break;
           tmem_ld_wait();
           const int cur = (c - c_begin) & 1;
@@ -990,7 +1020,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty0_leader + static_cast<uint32_t>(acc) * 8u);
-      if (++acc == NUM_ACC) { acc = 0; acc_phase ^= 1u; }
+      if (++acc == C::NUM_ACC) { acc = 0; acc_phase ^= 1u; }
       if (in_region && !red_tile) partial_signal(a, ctr, lane);
     }
     if (lane == 0) bulk_wait_group_all();  // our output stores are complete before exit
@@ -1018,7 +1048,21 @@ static bool gemm_use_pairs() {
   return v == 1;
 }
 
+// 256 x 512 pair tiles (TPB_GEMM_WIDE=0 turns them off) for the grids they bring down to
+// one round of tiles.
+static bool gemm_use_wide() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("TPB_GEMM_WIDE");
+    v = (e && e[0] == '0') ? 0 : 1;
+  }
+  return v == 1;
+}
+
 typedef void (*GemmKernel)(GemmArgs);
+
+// Kernel variants: the one-CTA kernel, CTA pairs on 256 x 256 tiles, CTA pairs on 256 x 512.
+enum { VAR_SINGLE = 0, VAR_PAIR = 1, VAR_PAIR_WIDE = 2, NUM_VAR = 3 };
 
 // The kernel instantiation for an epilogue kind and operand layout: each instantiation holds
 // only its own epilogue and operand addressing, so neither the register budget nor the
@@ -1026,9 +1070,16 @@ typedef void (*GemmKernel)(GemmArgs);
 // library launches: forward layers (K-major A, N-major B) with every forward epilogue; the
 // backward's dZ (K-major B, fp16 factor), weight gradients (M-major A, fp32 out) and dX
 // (K-major B, sum over shards).
-static GemmKernel gemm_kernel_for(int epi, int opl, bool pair) {
+static GemmKernel gemm_kernel_for(int epi, int opl, int var) {
+  // wide tiles: the row layer's bias + residual epilogue (forward, and the backward's dX)
+  if (var == VAR_PAIR_WIDE) {
+    if (epi == EPI_BIAS_RESID && opl == 0) return tp_gemm_pair_kernel<EPI_BIAS_RESID, 0, 512>;
+    if (epi == EPI_BIAS_RESID && opl == OPL_B_KMAJOR) return tp_gemm_pair_kernel<EPI_BIAS_RESID, OPL_B_KMAJOR, 512>;
+    return nullptr;
+  }
+  const bool pair = var == VAR_PAIR;
 #define TP_GEMM_PICK(E, O) \
-  if (epi == E && opl == O) return pair ? tp_gemm_pair_kernel<E, O> : tp_gemm_kernel<E, O>;
+  if (epi == E && opl == O) return pair ? tp_gemm_pair_kernel<E, O, 256> : tp_gemm_kernel<E, O>;
   TP_GEMM_PICK(EPI_ACT, 0)
   TP_GEMM_PICK(EPI_PARTIAL_F32, 0)
   TP_GEMM_PICK(EPI_BIAS_RESID, 0)
@@ -1046,18 +1097,18 @@ static int operand_layout(const GemmArgs& a) { return (a.a_mn ? OPL_A_MN : 0) | 
 
 constexpr int NUM_EPI = 6;
 static int g_pair_clusters[64] = {0};
-static bool g_attr_set[64][2][NUM_EPI][4] = {};
+static bool g_attr_set[64][NUM_VAR][NUM_EPI][4] = {};
 
 // Allow the kernel's dynamic shared memory (once per device and instantiation).
-static tp_status set_smem_attr(int dev, int epi, int opl, bool pair) {
+static tp_status set_smem_attr(int dev, int epi, int opl, int var) {
   const bool known = dev >= 0 && dev < 64 && epi >= 0 && epi < NUM_EPI && opl >= 0 && opl < 4;
-  if (known && g_attr_set[dev][pair][epi][opl]) return TP_OK;
-  GemmKernel k = gemm_kernel_for(epi, opl, pair);
+  if (known && g_attr_set[dev][var][epi][opl]) return TP_OK;
+  GemmKernel k = gemm_kernel_for(epi, opl, var);
   if (!k) return set_error(TP_ERR_CUDA, "no GEMM instantiation for this epilogue and operand layout");
-  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pair ? P_SMEM_BYTES : SMEM_BYTES) !=
-      cudaSuccess)
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           var == VAR_SINGLE ? SMEM_BYTES : P_SMEM_BYTES) != cudaSuccess)
     return set_error(TP_ERR_CUDA, "cudaFuncSetAttribute (shared memory) failed");
-  if (known) g_attr_set[dev][pair][epi][opl] = true;
+  if (known) g_attr_set[dev][var][epi][opl] = true;
   return TP_OK;
 }
 
@@ -1066,7 +1117,7 @@ static tp_status set_smem_attr(int dev, int epi, int opl, bool pair) {
 static int pair_clusters(int dev) {
   if (dev < 0 || dev >= 64) return 0;
   if (g_pair_clusters[dev]) return g_pair_clusters[dev];
-  if (set_smem_attr(dev, EPI_ACT, 0, true) != TP_OK) return -1;
+  if (set_smem_attr(dev, EPI_ACT, 0, VAR_PAIR) != TP_OK) return -1;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1079,7 +1130,7 @@ static int pair_clusters(int dev) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_kernel_for(EPI_ACT, 0, true), &cfg) != cudaSuccess || n <= 0) return -1;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_kernel_for(EPI_ACT, 0, VAR_PAIR), &cfg) != cudaSuccess || n <= 0) return -1;
   g_pair_clusters[dev] = n;
   return n;
 }
@@ -1088,15 +1139,27 @@ static tp_status launch_gemm_pair(const GemmArgs& a, cudaStream_t stream, const 
   const int nclusters_max = pair_clusters(dev);
   if (nclusters_max <= 0) return TP_ERR_CUDA;
   const int opl = operand_layout(a);
-  const tp_status sa = set_smem_attr(dev, a.epi, opl, true);
-  if (sa != TP_OK) return sa;
   const int m_tiles = (a.M + P_ROWS - 1) / P_ROWS;
-  const int n_tiles = (a.N + BN - 1) / BN;
-  const long long tiles = 1LL * m_tiles * n_tiles * (a.concat ? 1 : a.G);
+  const long long tiles256 = 1LL * m_tiles * ((a.N + 255) / 256) * (a.concat ? 1 : a.G);
+  const long long tiles512 = 1LL * m_tiles * ((a.N + 511) / 512) * (a.concat ? 1 : a.G);
+  // A wide tile is twice the tensor work of a 256 x 256 one, with a quarter fewer operand
+  // bytes per SM, but its one accumulator leaves each round's epilogue exposed.  So: wide
+  // where that takes no more rounds of tensor work (2 * rounds512 <= rounds256) and either
+  // one round suffices or the K loop is long enough (>= 128 steps of 64) for the exposed
+  // epilogue to be a few percent of a round.
+  const long long rounds256 = (tiles256 + nclusters_max - 1) / nclusters_max;
+  const long long rounds512 = (tiles512 + nclusters_max - 1) / nclusters_max;
+  const long long k_steps = 1LL * ((a.Kg + BK - 1) / BK) * (a.concat ? a.G : 1);
+  const bool wide = gemm_use_wide() && gemm_kernel_for(a.epi, opl, VAR_PAIR_WIDE) != nullptr &&
+                    2 * rounds512 <= rounds256 && (rounds512 == 1 || k_steps >= 128);
+  const int var = wide ? VAR_PAIR_WIDE : VAR_PAIR;
+  const tp_status sa = set_smem_attr(dev, a.epi, opl, var);
+  if (sa != TP_OK) return sa;
+  const long long tiles = wide ? tiles512 : tiles256;
   if (tiles <= 0) return TP_OK;
   const int nclusters = static_cast<int>(tiles < nclusters_max ? tiles : nclusters_max);
   trace_before(stream, name);
-  const tp_status st = launch_ex(gemm_kernel_for(a.epi, opl, true), dim3(2 * nclusters), dim3(THREADS), P_SMEM_BYTES,
+  const tp_status st = launch_ex(gemm_kernel_for(a.epi, opl, var), dim3(2 * nclusters), dim3(THREADS), P_SMEM_BYTES,
                                  stream, 2, a);
   if (st != TP_OK) return st;
   trace_after(stream, name);
@@ -1108,7 +1171,7 @@ tp_status launch_gemm(const GemmArgs& a, cudaStream_t stream, const char* name) 
   if (cudaGetDevice(&dev) != cudaSuccess) return TP_ERR_CUDA;
   if (gemm_use_pairs()) return launch_gemm_pair(a, stream, name, dev);
   const int opl = operand_layout(a);
-  const tp_status sa = set_smem_attr(dev, a.epi, opl, false);
+  const tp_status sa = set_smem_attr(dev, a.epi, opl, VAR_SINGLE);
   if (sa != TP_OK) return sa;
   const int m_tiles = (a.M + BM - 1) / BM;
   const int n_tiles = (a.N + BN - 1) / BN;
@@ -1116,7 +1179,7 @@ tp_status launch_gemm(const GemmArgs& a, cudaStream_t stream, const char* name) 
   if (tiles <= 0) return TP_OK;
   const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
   trace_before(stream, name);
-  const tp_status st = launch_ex(gemm_kernel_for(a.epi, opl, false), dim3(grid), dim3(THREADS), SMEM_BYTES, stream, 1, a);
+  const tp_status st = launch_ex(gemm_kernel_for(a.epi, opl, VAR_SINGLE), dim3(grid), dim3(THREADS), SMEM_BYTES, stream, 1, a);
   if (st != TP_OK) return st;
   trace_after(stream, name);
   return TP_OK;

@@ -65,6 +65,16 @@ def test_bf16_small_full(M, h, f, t, mode, w2_fp16):
     assert_bf16_close(out, _oracle_full(inp), f"M{M} h{h} f{f} t{t} {mode} w2_fp16={w2_fp16}")
 
 
+@pytest.mark.parametrize("t", [1, 2])
+def test_bf16_wide_hidden_full(t):
+    """h = 10176 with M = 300: the row layer's 256 x 256 tiles (80) outnumber the CTA pairs and
+    its 256 x 512 tiles (40, the last one 448 columns wide) do not, so it runs on the wide
+    tiles; every element against the oracle."""
+    inp = inputs.ffn_inputs(300, 10176, 256, "bf16", seed=4, device=DEV)
+    out = _run_ffn(inp, t)
+    assert_bf16_close(out, _oracle_full(inp), f"M300 h10176 f256 t{t}")
+
+
 def test_bf16_relu_and_no_bias():
     inp = inputs.ffn_inputs(200, 256, 1024, "bf16", seed=2, device=DEV)
     out = _run_ffn(inp, 2, act="relu")
@@ -142,10 +152,12 @@ def test_row_linear(mode):
     assert_bf16_close(out, ref, f"row linear {mode}")
 
 
-# Wide fused row layers, every element checked: two blocks of 256 rows x 40 column tiles
-# (more tiles than CTA pairs, a second round of tiles), ragged M, and N = 10176, which is
-# not a multiple of the 256-column tile.
-ROW_WIDE_CASES = [(512, 256, 10240, 2), (300, 128, 10176, 1), (400, 512, 10240, 4)]
+# Wide fused row layers, every element checked.  Two blocks of 256 rows x 40 column tiles
+# of 256 are more tiles than CTA pairs, so these run on 256 x 512 tiles in one round (with
+# TPB_GEMM_WIDE=0: 256 x 256 tiles in two rounds); four blocks of rows (1024) are more
+# 256 x 512 tiles than pairs too and run on 256 x 256 tiles in three rounds.  Ragged M,
+# and N = 10176, which is a multiple of neither tile width.
+ROW_WIDE_CASES = [(512, 256, 10240, 2), (300, 128, 10176, 1), (400, 512, 10240, 4), (1024, 128, 10176, 2)]
 
 
 @pytest.mark.parametrize("M,k,n,t", ROW_WIDE_CASES)
@@ -164,7 +176,32 @@ def test_row_linear_wide_full(M, k, n, t):
     assert_bf16_close(out, ref, f"row linear {M}x{k}x{n} t={t}")
 
 
-ROW_PARTIAL_CASES = [(300, 384, 4), (1, 320, 2), (129, 256, 1), (513, 1024, 8), (2048, 4096, 4)]
+def test_row_linear_wide_two_rounds_sampled():
+    """M = 3684 (15 blocks of 256 rows, the last ragged), N = 4096, K = 8192 over t = 2: 120
+    tiles of 256 x 512 take two rounds of the CTA pairs (240 tiles of 256 x 256 would take
+    four), with 128 K steps per tile, so the row layer runs on wide tiles with an exposed
+    epilogue between rounds.  Eight rows of every block of rows, every column, against the
+    oracle; every element finite."""
+    M, k, n, t = 3684, 8192, 4096, 2
+    g = torch.Generator(device=DEV).manual_seed(17)
+    A = torch.randn(M, k, generator=g, device=DEV).to(torch.bfloat16)
+    W = (torch.randn(k, n, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    bias = (torch.randn(n, generator=g, device=DEV) * 0.01).to(torch.bfloat16)
+    R = torch.randn(M, n, generator=g, device=DEV).to(torch.bfloat16)
+    out = torch.full((M, n), float("nan"), dtype=torch.bfloat16, device=DEV)
+    tb.tp_row_linear_forward(A, tb.shard_rows(W, t), bias, R, out, mode="fused")
+    assert tb.tp_get_device_status() == tb.TP_OK
+    assert torch.isfinite(out.float()).all(), "an output element was not written"
+    rng = np.random.default_rng(17)
+    rows = np.concatenate([b + rng.choice(min(256, M - b), 8, replace=False) for b in range(0, M, 256)])
+    rows_t = torch.as_tensor(rows, device=DEV)
+    A_s, R_s = A[rows_t], R[rows_t]
+    ref = oracle.reduce_partials([to64(A_s[:, i * k // t:(i + 1) * k // t]) @ to64(W[i * k // t:(i + 1) * k // t])
+                                  for i in range(t)], to64(bias), to64(R_s))
+    assert_bf16_close(out[rows_t], ref, f"row linear {M}x{k}x{n} t={t}, {len(rows)} sampled rows")
+
+
+ROW_PARTIAL_CASES =[(300, 384, 4), (1, 320, 2), (129, 256, 1), (513, 1024, 8), (2048, 4096, 4)]
 
 
 def _row_partials_case(M, n, t):
