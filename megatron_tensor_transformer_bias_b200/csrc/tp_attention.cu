@@ -60,6 +60,18 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
       : "memory");
 }
 
+// mma_f16_ts issued by the lane elect.sync picks (whole warp converged).
+__device__ __forceinline__ void mma_f16_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, uint64_t* bar, int32_t x, int32_t y,
                                             int32_t z) {
   asm volatile(
@@ -607,8 +619,9 @@ __global__ void __launch_bounds__(tt::THREADS, 1) tp_attention_tt_kernel(const _
         mbar_wait_bounded(&k_full[j & 1], (j >> 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
       for (int j = max(0, nv - 2); j < nv; ++j)
         mbar_wait_bounded(&v_full[j & 1], (j >> 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
-    } else if (warp == 9 && lane == 0) {
+    } else if (warp == 9) {
       // ------------------------------------------------------------ MMA issuer
+      // The whole warp runs the loop (its values stay warp-uniform); one elected lane issues.
       // Shared-memory descriptors of every operand buffer, built once: an MMA's operand is
       // its buffer's descriptor plus the byte offset / 16 in the start-address field (the
       // field holds address / 16 in 14 bits; no buffer ends above 256 KB, so no carry).
@@ -636,11 +649,11 @@ __global__ void __launch_bounds__(tt::THREADS, 1) tp_attention_tt_kernel(const _
               // item's epilogue must have read out
               const int jp = j - 1;
               const int gv = gb + jp;
-              if (!mbar_wait_bounded(&p_full[t], (blk[t] + jp) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN) ||
+              if (!warp_wait_bounded(&p_full[t], (blk[t] + jp) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN) ||
                   (jp == 0 && nq[t] > 0 &&
-                   !mbar_wait_bounded(&o_empty[t], (nq[t] - 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN)) ||
+                   !warp_wait_bounded(&o_empty[t], (nq[t] - 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN)) ||
                   (!v_ready &&
-                   !mbar_wait_bounded(&v_full[gv & 1], (gv >> 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN))) {
+                   !warp_wait_bounded(&v_full[gv & 1], (gv >> 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN))) {
                 ok = false;
                 break;
               }
@@ -650,16 +663,16 @@ __global__ void __launch_bounds__(tt::THREADS, 1) tp_attention_tt_kernel(const _
               const uint32_t t_o = tmem_base + tt::O_COL + static_cast<uint32_t>(t * D);
 #pragma unroll
               for (int kk = 0; kk < tt::BK / 16; ++kk)
-                mma_f16_ts(t_o, t_s + static_cast<uint32_t>(kk * 8), vd + static_cast<uint64_t>((kk * 16 * 128) >> 4),
+                mma_f16_ts_elect(t_o, t_s + static_cast<uint32_t>(kk * 8), vd + static_cast<uint64_t>((kk * 16 * 128) >> 4),
                            tt::IDESC_PV, (jp > 0 || kk > 0) ? 1u : 0u);
-              if (j == it.n[t]) mma_commit(&o_done[t]);
+              if (j == it.n[t]) mma_commit_elect(&o_done[t]);
             }
             if (j < it.n[t]) {
               // S_t,j = Q_t K_j^T
               if ((j == 0 &&
-                   !mbar_wait_bounded(&q_full[t], nq[t] & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN)) ||
+                   !warp_wait_bounded(&q_full[t], nq[t] & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN)) ||
                   (!k_ready &&
-                   !mbar_wait_bounded(&k_full[gj & 1], (gj >> 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN))) {
+                   !warp_wait_bounded(&k_full[gj & 1], (gj >> 1) & 1, a.wait_limit_ns, a.status, WAIT_SITE_ATTN))) {
                 ok = false;
                 break;
               }
@@ -671,16 +684,16 @@ __global__ void __launch_bounds__(tt::THREADS, 1) tp_attention_tt_kernel(const _
               for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t off_q = (kk >> 2) * tt::Q_HALF + (kk & 3) * 32;
                 const uint32_t off_k = (kk >> 2) * tt::KV_HALF + (kk & 3) * 32;
-                mma_bf16_ss(t_s, qd + static_cast<uint64_t>(off_q >> 4), kd + static_cast<uint64_t>(off_k >> 4),
+                mma_bf16_ss_elect(t_s, qd + static_cast<uint64_t>(off_q >> 4), kd + static_cast<uint64_t>(off_k >> 4),
                             tt::IDESC_S, kk > 0 ? 1u : 0u);
               }
-              mma_commit(&s_full[t]);
-              if (j == it.n[t] - 1) mma_commit(&q_empty[t]);
+              mma_commit_elect(&s_full[t]);
+              if (j == it.n[t] - 1) mma_commit_elect(&q_empty[t]);
             }
           }
           if (!ok) break;
-          if (j >= 1) mma_commit(&v_empty[(gj - 1) & 1]);
-          if (j < it.n_max) mma_commit(&k_empty[gj & 1]);
+          if (j >= 1) mma_commit_elect(&v_empty[(gj - 1) & 1]);
+          if (j < it.n_max) mma_commit_elect(&k_empty[gj & 1]);
         }
 #pragma unroll
         for (int t = 0; t < 2; ++t)
@@ -691,8 +704,8 @@ __global__ void __launch_bounds__(tt::THREADS, 1) tp_attention_tt_kernel(const _
         gb += it.n_max;
       }
       if (!ok) *abort_flag = 1;
-      mma_commit(drain_bar);
-      mbar_wait_bounded(drain_bar, 0, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
+      mma_commit_elect(drain_bar);
+      warp_wait_bounded(drain_bar, 0, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
     }
   } else {
     // ------------------------------------------------------------ softmax + output of tile t

@@ -66,12 +66,14 @@ constexpr int DQ_SMEM = 1024 + 2 * TILE_R + NST_Q * STAGE_Q + STAGING + 256;
 // TMEM: score buffer b at b*128 (64 columns), its dP at b*128 + 64; accumulators at 256 (and 384)
 constexpr uint32_t T_ACC0 = 256, T_ACC1 = 384;
 
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
+// D[tmem] (+)= A[tmem] * B[smem desc], issued by the lane elect.sync picks (whole warp converged).
+__device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -117,18 +119,20 @@ __device__ __forceinline__ uint64_t nmajor_desc(uint32_t base, int kk) {
 }
 
 // D[128 x 64] = A[resident 128 x d] * B[streamed 64 x d]^T, both K-major in shared memory.
+// Issued by an issuing warp (all lanes converged; one elected lane issues).
 __device__ __forceinline__ void mma_ss_tile(uint32_t d_tmem, uint32_t a_base, uint32_t b_base) {
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk)
-    mma_bf16_ss(d_tmem, kmajor_desc(a_base, kk, HALF_R), kmajor_desc(b_base, kk, HALF_S), IDESC_SS,
+    mma_bf16_ss_elect(d_tmem, kmajor_desc(a_base, kk, HALF_R), kmajor_desc(b_base, kk, HALF_S), IDESC_SS,
                 kk > 0 ? 1u : 0u);
 }
 
-// D[128 x d] (+)= A[tmem, 128 x 64 fp16] * B[streamed 64 x d, read N-major].
+// D[128 x d] (+)= A[tmem, 128 x 64 fp16] * B[streamed 64 x d, read N-major].  Issued by an
+// issuing warp (all lanes converged; one elected lane issues).
 __device__ __forceinline__ void mma_ts_tile(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base, bool accumulate) {
 #pragma unroll
   for (int kk = 0; kk < BS / 16; ++kk)
-    mma_ts(d_tmem, a_tmem + static_cast<uint32_t>(kk * 8), nmajor_desc(b_base, kk), IDESC_TS,
+    mma_ts_elect(d_tmem, a_tmem + static_cast<uint32_t>(kk * 8), nmajor_desc(b_base, kk), IDESC_TS,
            (accumulate || kk > 0) ? 1u : 0u);
 }
 
@@ -263,10 +267,14 @@ __device__ __forceinline__ void bwd_bars_init(const BwdBars& z, int ts_issuers) 
 __device__ __forceinline__ bool bwait(uint64_t* bar, uint32_t parity, const AttnBwdArgs& a) {
   return mbar_wait_bounded(bar, parity, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
 }
+// The same wait taken by a whole issuing warp (one verdict for all lanes).
+__device__ __forceinline__ bool bwait_warp(uint64_t* bar, uint32_t parity, const AttnBwdArgs& a) {
+  return warp_wait_bounded(bar, parity, a.wait_limit_ns, a.status, WAIT_SITE_ATTN);
+}
 
-// One MMA-issuing thread's work on one item.  Each kernel has two such threads with disjoint
-// products: a single thread issues an MMA every ~100 cycles whatever its size, half the tensor
-// pipe's rate on these 64-wide tiles.  `issue_ss(n, g)` is this thread's score product of the
+// One MMA-issuing warp's work on one item (all 32 lanes run it; one elected lane issues).
+// Each kernel has two such warps with disjoint products: a single issuer issues an MMA every
+// ~50-100 cycles whatever its size, below the tensor pipe's rate on these 64-wide tiles.  `issue_ss(n, g)` is this thread's score product of the
 // item's sub-block n (running sub-block g, into score buffer g & 1), `issue_ts(n, g)` its
 // gradient product (when `has_ts`), issued once the compute warps have written P and dS of
 // g.  A score product into a buffer waits until the compute warps are done with the buffer's
@@ -282,13 +290,13 @@ __device__ __forceinline__ bool issue_item(int N, int g0, int item, const BwdBar
                                            bool has_ts, SS issue_ss, TS issue_ts) {
   auto score = [&](int n) -> bool {
     const int g = g0 + n;
-    if (g >= 2 && !bwait(&z.p_full[g & 1], ((g - 2) >> 1) & 1, a)) return false;
-    if (!bwait(&z.st_full[g % NSTG], (g / NSTG) & 1, a)) return false;
+    if (g >= 2 && !bwait_warp(&z.p_full[g & 1], ((g - 2) >> 1) & 1, a)) return false;
+    if (!bwait_warp(&z.st_full[g % NSTG], (g / NSTG) & 1, a)) return false;
     tc_fence_after();
     issue_ss(n, g);
-    mma_commit(&z.s_full[g & 1]);
-    if (!has_ts) mma_commit(&z.st_empty[g % NSTG]);
-    if (n == N - 1) mma_commit(z.res_empty);
+    mma_commit_elect(&z.s_full[g & 1]);
+    if (!has_ts) mma_commit_elect(&z.st_empty[g % NSTG]);
+    if (n == N - 1) mma_commit_elect(z.res_empty);
     return true;
   };
   for (int n = 0; n < N && n < 2; ++n)
@@ -296,15 +304,15 @@ __device__ __forceinline__ bool issue_item(int N, int g0, int item, const BwdBar
   for (int n = 0; n < N; ++n) {
     const int g = g0 + n;
     if (has_ts) {
-      if (!bwait(&z.p_full[g & 1], (g >> 1) & 1, a)) return false;
-      if (n == 0 && item > 0 && !bwait(z.acc_empty, (item - 1) & 1, a)) return false;
+      if (!bwait_warp(&z.p_full[g & 1], (g >> 1) & 1, a)) return false;
+      if (n == 0 && item > 0 && !bwait_warp(z.acc_empty, (item - 1) & 1, a)) return false;
       tc_fence_after();
       issue_ts(n, g);
-      mma_commit(&z.st_empty[g % NSTG]);
+      mma_commit_elect(&z.st_empty[g % NSTG]);
     }
     if (n + 2 < N && !score(n + 2)) return false;
   }
-  if (has_ts) mma_commit(z.acc_full);
+  if (has_ts) mma_commit_elect(z.acc_full);
   return true;
 }
 
@@ -439,7 +447,8 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attn_bwd_dkdv_kernel(const __gr
   } else if (warp <= ISSUERS) {
     // issuer 0: S^T = K Q_n^T and dV += P^T dO_n (buffer columns 0..63);
     // issuer 1: dP^T = V dO_n^T and dK += dS^T Q_n (buffer columns 64..127)
-    if (lane == 0) {
+    // (the whole warp runs the loop; one elected lane issues)
+    {
       const uint32_t col = static_cast<uint32_t>((warp - 1) * 64);
       const uint32_t resA = smem_u32(warp == 1 ? sK : sV);
       const uint32_t ss_off = warp == 1 ? 0u : static_cast<uint32_t>(TILE_S);    // Q_n or dO_n
@@ -450,7 +459,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attn_bwd_dkdv_kernel(const __gr
       for (int r = 0; r < rounds && ok; ++r) {
         BwdItem it;
         if (!bwd_item(a, r, true, it)) continue;
-        ok = bwait(z.res_full, item & 1, a);
+        ok = bwait_warp(z.res_full, item & 1, a);
         if (ok) {
           tc_fence_after();
           ok = issue_item<NST_KV>(
@@ -470,8 +479,8 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attn_bwd_dkdv_kernel(const __gr
         ++item;
       }
       if (!ok) *abort_flag = 1;
-      mma_commit(z.drain);
-      bwait(z.drain, 0, a);
+      mma_commit_elect(z.drain);
+      bwait_warp(z.drain, 0, a);
     }
   } else {
     // one key row per thread
@@ -645,7 +654,8 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attn_bwd_dq_kernel(const __grid
     }
   } else if (warp <= ISSUERS) {
     // issuer 0: S = Q K_n^T and dQ += dS K_n (buffer columns 0..63); issuer 1: dP = dO V_n^T
-    if (lane == 0) {
+    // (the whole warp runs the loop; one elected lane issues)
+    {
       const uint32_t col = static_cast<uint32_t>((warp - 1) * 64);
       const uint32_t resA = smem_u32(warp == 1 ? sQ : sdO);
       const uint32_t ss_off = warp == 1 ? 0u : static_cast<uint32_t>(TILE_S);    // K_n or V_n
@@ -654,7 +664,7 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attn_bwd_dq_kernel(const __grid
       for (int r = 0; r < rounds && ok; ++r) {
         BwdItem it;
         if (!bwd_item(a, r, false, it)) continue;
-        ok = bwait(z.res_full, item & 1, a);
+        ok = bwait_warp(z.res_full, item & 1, a);
         if (ok) {
           tc_fence_after();
           ok = issue_item<NST_Q>(
@@ -674,8 +684,8 @@ __global__ void __launch_bounds__(THREADS, 1) tp_attn_bwd_dq_kernel(const __grid
         ++item;
       }
       if (!ok) *abort_flag = 1;
-      mma_commit(z.drain);
-      bwait(z.drain, 0, a);
+      mma_commit_elect(z.drain);
+      bwait_warp(z.drain, 0, a);
     }
   } else {
     // one query row per thread

@@ -897,7 +897,8 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader only)
-    if (lane == 0 && leader) {
+    // The whole warp runs the loop (its values stay warp-uniform); one elected lane issues.
+    if (leader) {
       const uint32_t idesc = a.ab_f16 ? idesc_f16_f32(P_ROWS, 256, A_MN, !B_KM)
                                       : idesc_bf16_f32(P_ROWS, 256, A_MN, !B_KM);
       const uint32_t sA_addr = smem_u32(sA);
@@ -908,14 +909,14 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int tile = cid; tile < num_tiles && ok; tile += nclusters) {
-        if (!mbar_wait_bounded(&acc_empty[acc], acc_phase ^ 1u, a.wait_limit_ns, a.status, WAIT_SITE_MMA_ACC)) {
+        if (!warp_wait_bounded(&acc_empty[acc], acc_phase ^ 1u, a.wait_limit_ns, a.status, WAIT_SITE_MMA_ACC)) {
           *abort_flag = 1; ok = false; break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * PBN);
         for (int it = 0; it < k_iters; ++it) {
-          if (*abort_flag) { ok = false; break; }
-          if (!mbar_wait_bounded(&full_bar[stage], phase, a.wait_limit_ns, a.status, WAIT_SITE_MMA_FULL)) {
+          if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
+          if (!warp_wait_bounded(&full_bar[stage], phase, a.wait_limit_ns, a.status, WAIT_SITE_MMA_FULL)) {
             *abort_flag = 1; ok = false; break;
           }
           tc_fence_after();
@@ -930,18 +931,18 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_pair_kernel(const __grid_c
               const uint32_t bh = b_base + static_cast<uint32_t>(h) * 16384u;
               const uint64_t bdesc = B_KM ? smem_desc_sw128(bh + k * 32, 16, 1024)
                                           : smem_desc_sw128(bh + k * 16 * 128, B_BLOCK_BYTES, 1024);
-              mma_pair_ss(d_tmem + static_cast<uint32_t>(h * 256), adesc, bdesc, idesc, (it > 0 || k > 0) ? 1u : 0u);
+              mma_pair_ss_elect(d_tmem + static_cast<uint32_t>(h * 256), adesc, bdesc, idesc, (it > 0 || k > 0) ? 1u : 0u);
             }
           }
-          mma_commit_pair_mask(&empty_bar[stage], 0x3);  // frees this stage in both CTAs
+          mma_commit_pair_mask_elect(&empty_bar[stage], 0x3);  // frees this stage in both CTAs
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        mma_commit_pair_mask(&acc_full[acc], 0x3);       // accumulator ready in both CTAs
+        mma_commit_pair_mask_elect(&acc_full[acc], 0x3);       // accumulator ready in both CTAs
         if (++acc == C::NUM_ACC) { acc = 0; acc_phase ^= 1u; }
       }
-      mma_commit_pair_local(drain_bar);
-      mbar_wait_bounded(drain_bar, 0, a.wait_limit_ns, a.status, WAIT_SITE_MMA_ACC);
+      mma_commit_pair_local_elect(drain_bar);
+      warp_wait_bounded(drain_bar, 0, a.wait_limit_ns, a.status, WAIT_SITE_MMA_ACC);
     }
   } else {
     // ------------------------------------------------------------ epilogue (warps 2..5 of both CTAs)
