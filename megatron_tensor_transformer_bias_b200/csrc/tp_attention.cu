@@ -428,9 +428,9 @@ __global__ void __launch_bounds__(THREADS, 2) tp_attention_kernel(const __grid_c
 //   warps 4..7   softmax and output of query tile 1
 //   warp 8       TMA: Q0 and Q1 per item, then K_j and V_j (two stages each, 128 keys per
 //                block) in one running sequence across items
-//   warp 9       TMEM allocation; one thread issues every MMA
+//   warp 9       TMEM allocation; issues every MMA (one lane elected per instruction)
 //   warps 10, 11 idle (they only hand their registers to the softmax warps)
-// Both tiles share each K/V block.  The MMA thread interleaves the tiles per key block:
+// Both tiles share each K/V block.  The MMA warp interleaves the tiles per key block:
 //   O0 += P0_{j-1} V_{j-1};  S0_j = Q0 K_j^T;  O1 += P1_{j-1} V_{j-1};  S1_j = Q1 K_j^T
 // so the tensor core works on one tile while the other tile's softmax runs.  Each score
 // row (128 keys) stays in registers: the softmax warpgroups raise their register limit
@@ -768,7 +768,7 @@ __global__ void __launch_bounds__(tt::THREADS, 1) tp_attention_tt_kernel(const _
         const bool move = mx > m_ref + RESCALE_LOG2;
         const float m_new = move ? mx : m_ref;
         // O_t is idle here: S_t,j was issued after O_t += P_t,{j-1} V_{j-1}, and its
-        // commit tracks every earlier MMA of the issuing thread.  Rescale it in place.
+        // commit tracks every earlier MMA of the issuing lane.  Rescale it in place.
         if (j > 0 && __any_sync(0xffffffffu, move)) {
           const float alpha = move ? exp2f(m_ref - m_new) : 1.0f;
 #pragma unroll 1
@@ -814,7 +814,7 @@ __global__ void __launch_bounds__(tt::THREADS, 1) tp_attention_tt_kernel(const _
         mbar_arrive(&p_full[t]);
       }
       if (!ok) break;
-      // epilogue: O_t / l to global, then hand O_t back to the MMA thread
+      // epilogue: O_t / l to global, then hand O_t back to the MMA warp
       if (!__all_sync(0xffffffffu, mbar_wait_bounded(&o_done[t], items & 1, a.wait_limit_ns, a.status,
                                                      WAIT_SITE_ATTN))) {
         ok = false;

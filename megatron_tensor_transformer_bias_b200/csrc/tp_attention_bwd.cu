@@ -50,7 +50,7 @@ constexpr int NST_KV = 3;                    // shared-memory stages of streamed
 constexpr int NST_Q = 4;                     // (dQ)
 constexpr int STAGING = 2 * HALF_R;          // a 128 x 128 bf16 gradient block on its way out (TMA store)
 constexpr int THREADS = 224;                 // warp 0 TMA, warps 1 and 2 MMA, warps 3..6 compute
-constexpr int ISSUERS = 2;                   // MMA-issuing threads (one MMA costs one thread ~100 cycles)
+constexpr int ISSUERS = 2;                   // MMA-issuing warps (an MMA costs its issuer ~50-100 cycles)
 constexpr int COMPUTE_THREADS = 128;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC_SS = idesc_f16_f32(BR, BS, 0, 0);   // resident x streamed^T, both K-major

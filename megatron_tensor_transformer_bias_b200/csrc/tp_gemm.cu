@@ -12,15 +12,18 @@
 // tile per (shard, m, n) writing fp32 partials.
 //
 // Two kernels share the roles below: tp_gemm_pair_kernel (the default; a cluster
-// of two CTAs computes a 256x256 tile with cta_group::2 MMAs) and tp_gemm_kernel
-// (one CTA, 128x256 tiles).  Roles per CTA (320 threads, one CTA per SM):
+// of two CTAs computes a 256x256 tile, or a 256x512 one, with cta_group::2 MMAs) and
+// tp_gemm_kernel (one CTA, 128x256 tiles).  Roles per CTA (320 threads, one CTA per SM):
 //   warp 0      TMA producer: this CTA's operand tiles, one 64-wide K step per stage
-//   warp 1      TMEM allocation; one thread issues tcgen05.mma (16-deep K per instruction)
+//   warp 1      TMEM allocation; issues tcgen05.mma (16-deep K per instruction): in the
+//               pair kernel the whole warp runs the loop and one lane is elected per
+//               instruction, in the one-CTA kernel lane 0 issues
 //   warps 2..9  epilogue: tcgen05.ld TMEM -> registers -> bias/act/residual -> global
 //               (16-bit outputs through swizzled shared-memory staging and TMA stores)
-// A shared-memory ring (6 stages for pairs, 4 for one CTA) feeds the MMA; two
-// 256-column TMEM accumulators let the epilogue of one tile overlap the main loop
-// of the next.
+// A shared-memory ring (6 stages of 32 KB for 256x256 pair tiles, 4 of 48 KB for 256x512,
+// 4 for one CTA) feeds the MMA; with 256-column tiles two TMEM accumulators let the
+// epilogue of one tile overlap the main loop of the next (a 256x512 tile's accumulator
+// fills all 512 columns).
 #include <cstdlib>
 
 #include "tp_internal.h"
@@ -1067,7 +1070,7 @@ enum { VAR_SINGLE = 0, VAR_PAIR = 1, VAR_PAIR_WIDE = 2, NUM_VAR = 3 };
 
 // The kernel instantiation for an epilogue kind and operand layout: each instantiation holds
 // only its own epilogue and operand addressing, so neither the register budget nor the
-// single MMA-issuing thread pays for the paths it does not take.  The combinations the
+// MMA-issuing warp pays for the paths it does not take.  The combinations the
 // library launches: forward layers (K-major A, N-major B) with every forward epilogue; the
 // backward's dZ (K-major B, fp16 factor), weight gradients (M-major A, fp32 out) and dX
 // (K-major B, sum over shards).
