@@ -76,10 +76,12 @@ typedef enum { TP_BF16 = 0, TP_FP32 = 1, TP_FP16 = 2 } tp_dtype;
  *                     (ascending or descending K, whichever starts on data
  *                     still in L2), and its epilogue adds the bias and the
  *                     residual.  The result is the same bits for every t.
- *                     A tile's place in the schedule depends on the number
- *                     of CTA pairs the device runs at once (74 on a 148-SM
- *                     B200), so the bits are reproducible across runs and
- *                     processes on devices with the same SM count.
+ *                     A tile's place in the schedule, and the tile width
+ *                     (256 or 512 columns, picked from the same count), depend
+ *                     on the number of CTA pairs the device runs at once (74
+ *                     on a 148-SM B200), so the bits are reproducible across
+ *                     runs and processes on devices with the same SM count
+ *                     (and the same TPB_GEMM_WIDE setting).
  * TP_REDUCE_PARTIALS: the row GEMM writes t fp32 partials Y_i [t, M, h] to the
  *                     workspace (TMA stores) and a reduce kernel sums them in
  *                     the order 0..t-1, then adds bias and residual.  With the
