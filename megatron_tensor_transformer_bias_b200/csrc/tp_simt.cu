@@ -241,8 +241,23 @@ __global__ void __launch_bounds__(256) colsum_kernel(const uint16_t* __restrict_
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   pdl_wait();
   if (c0 < n) {
-#pragma unroll 4
-    for (int64_t r = r_lo + slot; r < r_hi; r += CS_SLOTS) {
+    // eight rows' loads in flight per thread (32 KB per CTA), then their adds in row order
+    int64_t r = r_lo + slot;
+    for (; r + 7 * CS_SLOTS < r_hi; r += 8 * CS_SLOTS) {
+      uint4 u[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) u[k] = __ldg(reinterpret_cast<const uint4*>(x + (r + k * CS_SLOTS) * ld + c0));
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          acc[2 * j] += __uint_as_float(w[j] << 16);
+          acc[2 * j + 1] += __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+      }
+    }
+    for (; r < r_hi; r += CS_SLOTS) {
       float f[8];
       load_bf16x8(x + r * ld + c0, f);
 #pragma unroll

@@ -54,9 +54,10 @@ def _oracle(inp, dY, act="gelu", with_b1=True, add_dY=True):
     return g
 
 
-# the last case's dX GEMM (N = h = 10176, two blocks of rows) runs on 256 x 512 tiles
+# (300, 10176, 256, 2): its dX GEMM (N = h = 10176, two blocks of rows) runs on 256 x 512 tiles;
+# (1100, 256, 512, 2): the column sums' batched eight-row loads and their one-row tail both run
 SMALL = [(300, 256, 1024, 4), (1, 64, 256, 2), (129, 128, 512, 1), (513, 512, 2048, 8), (64, 192, 384, 3),
-         (300, 10176, 256, 2)]
+         (300, 10176, 256, 2), (1100, 256, 512, 2)]
 
 
 @pytest.mark.parametrize("M,h,f,t", SMALL)
