@@ -728,12 +728,11 @@ __global__ void __launch_bounds__(THREADS, 1) tp_gemm_kernel(const __grid_consta
 // barriers; both CTAs' epilogues arrive on the leader's accumulator-empty barrier.
 // No load is multicast.
 //
-// A wide variant (PBN = 512: 256 x 512 tiles) serves grids whose 256 x 256 tiles would
-// take more than one round but whose 256 x 512 tiles fit in one: each 64-wide K step
-// feeds two N=256 MMAs from one A tile, so an SM streams 48 KB per 1024 tensor cycles
-// instead of 32 KB per 512 (a quarter fewer operand bytes for the same work).  Its one
-// accumulator fills all 512 TMEM columns (no epilogue/main-loop overlap across tiles,
-// which a one-round grid does not have).
+// A wide variant (PBN = 512: 256 x 512 tiles): each 64-wide K step feeds two N=256 MMAs
+// from one A tile, so an SM streams 48 KB per 1024 tensor cycles instead of 32 KB per 512
+// (a quarter fewer operand bytes for the same work).  Its one accumulator fills all 512
+// TMEM columns, so each round's epilogue is exposed instead of overlapping the next tile's
+// main loop; the launcher picks it only where that costs little (launch_gemm_pair).
 constexpr int P_ROWS = 2 * BM;                      // 256 rows per pair
 constexpr int P_A_BYTES = BM * BK * 2;              // 16 KB per CTA
 
